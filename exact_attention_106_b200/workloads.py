@@ -1,0 +1,123 @@
+"""Seeded synthetic workloads for exact attention.
+
+This module only draws random inputs and names the problem shapes; it holds
+none of the attention arithmetic.  Both the CUDA path and the fp64 oracle are
+fed from here, so that they see the very same bf16 values.
+
+Recipe (shared by tests and the benchmark):
+  * every tensor is drawn as float32 i.i.d. N(0, 1) with a CPU
+    ``torch.Generator`` seeded per tensor, then rounded to bfloat16
+    (round-to-nearest-even, torch's cast);
+  * seeds: Q = base + 0, K = base + 1, V = base + 2, dO = base + 3, where
+    ``base`` is 1000 x (workload number) plus 100 x (sweep point number);
+  * layout is contiguous ``[B, H, N, d]``, the (batch, heads, seq_len,
+    head_dim) order of the PyTorch example in "11.11 Flash Attention",
+    §Using Flash Attention, and of the (B, N_h, T, D_h) shapes in
+    "Flash Attention: From Theory to Implementation", introduction;
+  * the "stability" workload multiplies Q by 8 on heads [H/2, H) of every
+    batch, in float32 before the bf16 cast (x8 is exact in bf16).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import List, Optional
+
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    causal: bool
+    seed_base: int
+    scale: Optional[float] = None      # None -> 1/sqrt(d)
+    q_boost_heads_from: Optional[int] = None  # heads h >= this get Q*8
+    q_boost: float = 8.0
+
+    @property
+    def softmax_scale(self) -> float:
+        return self.scale if self.scale is not None else 1.0 / math.sqrt(self.d)
+
+    @property
+    def shape(self):
+        return (self.B, self.H, self.N, self.d)
+
+    def pairs(self) -> int:
+        """Unmasked (query, key) pairs: the algorithmic work unit."""
+        per_head = self.N * (self.N + 1) // 2 if self.causal else self.N * self.N
+        return self.B * self.H * per_head
+
+    def fwd_flops(self) -> int:
+        """Two matmuls (QK^T and PV) of 2*d flops per unmasked pair."""
+        return 4 * self.d * self.pairs()
+
+    def bwd_flops(self) -> int:
+        """Five matmuls: the recomputed QK^T plus dV, dP, dQ and dK."""
+        return 10 * self.d * self.pairs()
+
+
+def _seeded_normal(shape, seed: int) -> torch.Tensor:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    return torch.randn(shape, generator=g, dtype=torch.float32)
+
+
+def make_inputs(w: Workload, with_grad_out: bool = True):
+    """Return (q, k, v, do) as contiguous CPU bfloat16 tensors [B,H,N,d]."""
+    q = _seeded_normal(w.shape, w.seed_base + 0)
+    if w.q_boost_heads_from is not None:
+        q[:, w.q_boost_heads_from:] *= w.q_boost
+    k = _seeded_normal(w.shape, w.seed_base + 1)
+    v = _seeded_normal(w.shape, w.seed_base + 2)
+    out = [q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)]
+    if with_grad_out:
+        out.append(_seeded_normal(w.shape, w.seed_base + 3).to(torch.bfloat16))
+    else:
+        out.append(None)
+    return tuple(out)
+
+
+# ---------------------------------------------------------------------------
+# The named workloads.  Sizes follow the shapes the pages use: head_dim 64/128,
+# 32 heads, sequence lengths from 512 to 32768.
+# ---------------------------------------------------------------------------
+TINY = Workload("tiny_1x1x128x64", 1, 1, 128, 64, False, 1000, scale=1.0 / 8.0)
+SMALL_CAUSAL_STABILITY = Workload("stability_2x8x1024x64_causal_q8", 2, 8, 1024, 64, True,
+                                  2000, q_boost_heads_from=4)
+LLAMA_BLOCK = Workload("llama_block_4x16x4096x128_causal", 4, 16, 4096, 128, True, 3000)
+LONG_CONTEXT = Workload("long_context_1x32x16384x128_causal", 1, 32, 16384, 128, True, 4000)
+
+NAMED = [TINY, SMALL_CAUSAL_STABILITY, LLAMA_BLOCK, LONG_CONTEXT]
+
+SWEEP_TOKENS = 16384
+SWEEP_N = [512, 1024, 2048, 4096, 8192, 16384]
+
+
+def sweep() -> List[Workload]:
+    """Fixed 16384 tokens per batch: B = 16384 / N, H = 32."""
+    out = []
+    idx = 0
+    for d in (64, 128):
+        for causal in (False, True):
+            for n in SWEEP_N:
+                idx += 1
+                out.append(Workload(
+                    f"sweep_{SWEEP_TOKENS // n}x32x{n}x{d}_{'causal' if causal else 'full'}",
+                    SWEEP_TOKENS // n, 32, n, d, causal, 5000 + 100 * idx))
+    return out
+
+
+SINGLE_HEAD_32K = Workload("single_head_1x1x32768x128_full", 1, 1, 32768, 128, False, 6000)
+SINGLE_HEAD_32K_CAUSAL = Workload("single_head_1x1x32768x128_causal", 1, 1, 32768, 128, True, 6100)
+
+
+def by_name(name: str) -> Workload:
+    for w in NAMED + sweep() + [SINGLE_HEAD_32K, SINGLE_HEAD_32K_CAUSAL]:
+        if w.name == name:
+            return w
+    raise KeyError(name)
