@@ -1,0 +1,380 @@
+"""Throughput of exact attention (forward + backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+A step is one forward and one backward pass (every stage of the path) over one
+batch of the long-context workload, B=1, H=32, N=16384, d=128, causal, bf16
+(seeded synthetic N(0,1) inputs; Q, K, V and dO are 128 MiB each, so every
+step's inputs are larger than the 126 MB L2).  Throughput is algorithmic
+TFLOP/s: 4*d flops per unmasked (query, key) pair for the forward, 10*d for the
+backward (five matmuls, one of them the recomputation of Q K^T).
+
+With N > 1 (launched by torch.distributed.run, one rank per GPU) every rank
+processes its own batch of that workload (weak scaling; no collective on the
+data path), and the reported time is the maximum over ranks.
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle on
+the host cores instead (a bounded sample of the same workload per step).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+METRIC = "attention fwd/bwd TFLOP/s (bf16, d=128, N 1k-32k) and % of B200 BF16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_bwd_dkdv_long_context_traffic.txt")
+KERNEL_SOURCES = [os.path.join(ROOT, "exact_attention_106_b200", "csrc", f)
+                  for f in ("bwd.cuh", "fwd.cuh", "ptx.cuh")]
+
+
+# --------------------------------------------------------------------- utils
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """Per-launch DRAM bytes of the backward main kernel from the committed ncu
+    summary, or None if absent or taken on a different kernel source."""
+    try:
+        kv = {}
+        with open(TRAFFIC_FILE) as f:
+            for line in f:
+                if ":" in line and not line.lstrip().startswith("#"):
+                    a, b = line.split(":", 1)
+                    kv[a.strip()] = b.strip()
+        if kv.get("kernel_source_sha256_16") != kernel_source_hash():
+            return None
+        return float(kv["traffic_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.out = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.gpu_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        if not self.out:
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def reduce_max(value: float, device) -> float:
+    """Maximum of a per-rank scalar over all ranks (identity without a process group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_workload(base, rank: int):
+    """Each rank gets its own batch: same shape, seeds shifted by the rank."""
+    import dataclasses
+    return dataclasses.replace(base, seed_base=base.seed_base + 10 * rank)
+
+
+# -------------------------------------------------------------- CPU baseline
+def oracle_sample(w, rows: int):
+    """The first `rows` tokens of head (0, 0) of workload w: under the causal
+    mask this is itself a complete attention problem of length `rows`."""
+    from exact_attention_106_b200 import workloads as W
+    import dataclasses
+    sub = dataclasses.replace(w, B=1, H=1, N=rows)
+    q, k, v, do = W.make_inputs(sub)
+    return sub, q, k, v, do
+
+
+def time_oracle(w, rows: int):
+    import oracle
+    sub, q, k, v, do = oracle_sample(w, rows)
+    t0 = time.perf_counter()
+    oracle.backward(q, k, v, do, sub.softmax_scale, sub.causal)
+    dt = time.perf_counter() - t0
+    return (sub.fwd_flops() + sub.bwd_flops()) / dt / 1e12, dt, sub
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return 1
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, rank, world, local_rank):
+    import exact_attention_106_b200 as ex
+    from exact_attention_106_b200 import workloads as W
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = rank_workload(W.by_name(args.workload), rank)
+    B, H, N, d = w.shape
+    q, k, v, do = W.make_inputs(w)
+    qd, kd, vd, dod = (x.to(dev) for x in (q, k, v, do))
+    o = torch.empty_like(qd)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = (torch.empty_like(qd) for _ in range(3))
+    ws = ex.alloc_workspace(B, H, N, d, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        ex.forward(qd, kd, vd, causal=w.causal, scale=w.softmax_scale, out=o, lse=lse)
+        if evs:
+            evs[1].record(stream)
+        for i, _ in enumerate(ex.bwd_stages(qd, kd, vd, o, lse, dod, dq, dk, dv, ws, causal=w.causal,
+                                            scale=w.softmax_scale)):
+            if evs:
+                evs[2 + i].record(stream)
+
+    import torch.distributed as dist
+    dist_on = dist.is_available() and dist.is_initialized()
+
+    def barrier():
+        if dist_on:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    if ex.device_status(dev) != 0:
+        raise RuntimeError("device status not clean after warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    with ClockSampler(local_rank) as clk:
+        t_start.record(stream)
+        for s in range(args.steps):
+            step(evs[s])
+        t_end.record(stream)
+        barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    status = ex.device_status(dev)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+    per_kernel = {name: [evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps)]
+                  for i, name in enumerate(["fwd", "bwd_preprocess", "bwd_dkdv", "bwd_dq_convert"])}
+    max_ms = reduce_max(elapsed_ms, dev)
+    flops_step = w.fwd_flops() + w.bwd_flops()
+
+    # e2e: pinned host buffers -> device -> fwd + bwd -> host, every step
+    hq, hk, hv, hdo = (x.pin_memory() for x in (q, k, v, do))
+    ho, hdq, hdk, hdv = (torch.empty(w.shape, dtype=torch.bfloat16).pin_memory() for _ in range(4))
+    hlse = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        for h, dv_ in ((hq, qd), (hk, kd), (hv, vd), (hdo, dod)):
+            dv_.copy_(h, non_blocking=True)
+        step()
+        for dv_, h in ((o, ho), (lse, hlse), (dq, hdq), (dk, hdk), (dv, hdv)):
+            h.copy_(dv_, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 20))
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    e2e_ms = reduce_max(e0.elapsed_time(e1), dev)
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hdo))
+    d2h = sum(x.numel() * x.element_size() for x in (ho, hlse, hdq, hdk, hdv))
+
+    if rank != 0:
+        return None
+    peaks, peak_src = load_peaks()
+    mean = {k_: statistics.mean(v_) for k_, v_ in per_kernel.items()}
+    fwd_tf = w.fwd_flops() / (mean["fwd"] * 1e-3) / 1e12
+    bwd_ms = mean["bwd_preprocess"] + mean["bwd_dkdv"] + mean["bwd_dq_convert"]
+    bwd_tf = w.bwd_flops() / (bwd_ms * 1e-3) / 1e12
+    dkdv_tf = w.bwd_flops() / (mean["bwd_dkdv"] * 1e-3) / 1e12
+    dominant = "bwd_dkdv" if mean["bwd_dkdv"] >= mean["fwd"] else "fwd"
+    dom_tf = dkdv_tf if dominant == "bwd_dkdv" else fwd_tf
+    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    value = world * flops_step * args.steps / (max_ms * 1e-3) / 1e12
+    rows = args.cpu_rows
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        v_cpu, dt_cpu, sub = time_oracle(w, rows)
+        cpu = {"value": v_cpu, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+               "seconds": dt_cpu,
+               "sample": f"fp64 numpy oracle, fwd+bwd of the first {rows} tokens of head (0,0) "
+                         f"(a complete causal problem 1x1x{rows}x{d}); algorithmic flops / time"}
+    spec_peak = 2250.0
+    result = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d, "causal": w.causal,
+                   "step": "forward + backward (all stages)", "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (Q, K, V, dO 128 MiB each per step)"},
+        "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
+        "pct_of_peak": {"fwd_of_measured_sustained": fwd_tf / peak, "bwd_of_measured_sustained": bwd_tf / peak,
+                        "fwd_of_spec_2250": fwd_tf / spec_peak, "bwd_of_spec_2250": bwd_tf / spec_peak,
+                        "peak_source": peak_src},
+        "kernels": {k_: {"mean_ms": mean[k_]} for k_ in mean},
+        "roofline": {"kernel": "attn_bwd_kernel<128>" if dominant == "bwd_dkdv" else "attn_fwd_kernel<128>",
+                     "bound": "tensor", "achieved": dom_tf, "peak": peak, "unit": "TFLOP/s",
+                     "frac": dom_tf / peak, "peak_kind": f"bf16 sustained ({peak_src})",
+                     "traffic": recorded_traffic() if dominant == "bwd_dkdv" else None},
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * flops_step * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "clocks": clk.summary(),
+        "gpu_launches": 4 * args.steps,
+    }
+    result["kernels"]["fwd"]["tflops"] = fwd_tf
+    result["kernels"]["bwd_dkdv"]["tflops"] = dkdv_tf
+    return result
+
+
+# ------------------------------------------------------------ reference arm
+def run_reference(args, rank):
+    from exact_attention_106_b200 import workloads as W
+    if rank != 0:
+        return None
+    w = W.by_name(args.workload)
+    rows = args.ref_rows
+    vals = []
+    for _ in range(args.warmup):
+        time_oracle(w, rows)
+    t_total = 0.0
+    for _ in range(args.steps):
+        v_, dt, sub = time_oracle(w, rows)
+        vals.append(v_)
+        t_total += dt
+    value = args.steps * (sub.fwd_flops() + sub.bwd_flops()) / t_total / 1e12
+    cores = blas_threads()
+    sample = (f"fp64 numpy oracle, fwd+bwd of the first {rows} tokens of head (0,0) of {w.name} "
+              f"(a complete causal problem 1x1x{rows}x{w.d}) per step")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+                   "step": "forward + backward", "sample_rows": rows},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="long_context_1x32x16384x128_causal")
+    ap.add_argument("--cpu-rows", type=int, default=4096, help="oracle sample size for cpu_baseline")
+    ap.add_argument("--ref-rows", type=int, default=2048, help="oracle sample size per reference step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+
+    if args.impl == "reference":
+        out = run_reference(args, rank)
+    else:
+        if world > 1:
+            import datetime
+            import torch.distributed as dist
+            torch.cuda.set_device(local_rank)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local_rank))
+        try:
+            out = run_ours(args, rank, world, local_rank)
+        finally:
+            import torch.distributed as dist
+            if dist.is_available() and dist.is_initialized():
+                dist.destroy_process_group()
+    if out is not None:
+        print(json.dumps(out), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

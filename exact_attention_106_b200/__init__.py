@@ -1,0 +1,113 @@
+"""exattn: exact scaled-dot-product attention on B200 (sm_100a).
+
+Python face of the C ABI in include/exattn.h.  Every function here only
+checks and marshals arguments (device pointers and the current CUDA stream)
+and calls the library; all arithmetic runs in its CUDA kernels.  PyTorch is
+used for device memory and streams.
+
+    o, lse = forward(q, k, v, causal=False, scale=None)
+    dq, dk, dv = backward(q, k, v, o, lse, do, causal=False, scale=None)
+
+Tensors are CUDA bfloat16, contiguous [B, H, N, d] with d in {64, 128};
+lse is float32 [B, H, N].  ``scale`` defaults to 1/sqrt(d).
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional
+
+import torch
+
+from . import _lib
+
+__all__ = ["forward", "backward", "bwd_workspace_bytes", "device_status", "ExattnError"]
+
+ExattnError = _lib.ExattnError
+
+
+def _stream(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check_qkv(*ts: torch.Tensor) -> None:
+    shape = ts[0].shape
+    for t in ts:
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous() and t.dim() == 4):
+            raise ValueError("expected contiguous CUDA bfloat16 tensors [B, H, N, d]")
+        if t.shape != shape or t.device != ts[0].device:
+            raise ValueError("q, k, v (and o, do) must share shape and device")
+
+
+def _scale(d: int, scale: Optional[float]) -> float:
+    return 1.0 / math.sqrt(d) if scale is None else float(scale)
+
+
+def forward(q, k, v, causal: bool = False, scale: Optional[float] = None, out=None, lse=None):
+    """O and per-row logsumexp of softmax(scale Q K^T) V."""
+    _check_qkv(q, k, v)
+    B, H, N, d = q.shape
+    o = torch.empty_like(q) if out is None else out
+    lse_t = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    lib = _lib.load()
+    _lib.check("attn_fwd", lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                        lse_t.data_ptr(), B, H, N, d, _scale(d, scale), int(causal),
+                                        _stream(q.device)))
+    return o, lse_t
+
+
+def bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(_lib.load().attn_bwd_workspace_bytes(B, H, N, d))
+
+
+def alloc_workspace(B: int, H: int, N: int, d: int, device) -> torch.Tensor:
+    """A device buffer for the backward (torch allocations are 256-byte aligned)."""
+    n = max(1, bwd_workspace_bytes(B, H, N, d))
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def backward(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] = None,
+             workspace: Optional[torch.Tensor] = None, out=None):
+    """dQ, dK, dV of sum(O * dO) for O = softmax(scale Q K^T) V."""
+    _check_qkv(q, k, v, o, do)
+    B, H, N, d = q.shape
+    if not (lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous() and lse.shape == (B, H, N)):
+        raise ValueError("lse must be contiguous CUDA float32 [B, H, N]")
+    if out is None:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    else:
+        dq, dk, dv = out
+    ws = alloc_workspace(B, H, N, d, q.device) if workspace is None else workspace
+    lib = _lib.load()
+    _lib.check("attn_bwd", lib.attn_bwd(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+        dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, _scale(d, scale), int(causal),
+        ws.data_ptr(), ws.numel(), _stream(q.device)))
+    return dq, dk, dv
+
+
+def bwd_stages(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool = False,
+               scale: Optional[float] = None):
+    """The backward as three separate C-ABI calls (what ``backward`` runs), each
+    returning after its launch; yields between stages so a caller can record
+    CUDA events around each."""
+    B, H, N, d = q.shape
+    sc = _scale(d, scale)
+    st = _stream(q.device)
+    lib = _lib.load()
+    _lib.check("attn_bwd_preprocess", lib.attn_bwd_preprocess(
+        o.data_ptr(), do.data_ptr(), lse.data_ptr(), B, H, N, d, workspace.data_ptr(), workspace.numel(), st))
+    yield "preprocess"
+    _lib.check("attn_bwd_dkdv", lib.attn_bwd_dkdv(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, sc,
+        int(causal), workspace.data_ptr(), workspace.numel(), st))
+    yield "dkdv"
+    _lib.check("attn_bwd_dq_convert", lib.attn_bwd_dq_convert(
+        dq.data_ptr(), B, H, N, d, sc, workspace.data_ptr(), workspace.numel(), st))
+    yield "dq_convert"
+
+
+def device_status(device=None) -> int:
+    """Synchronise the current stream and return (and clear) the device status word."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        return int(_lib.load().attn_get_device_status(_stream(dev)))

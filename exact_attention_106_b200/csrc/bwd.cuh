@@ -1,0 +1,490 @@
+// Backward kernels.  The forward keeps only Q, K, V, O and the per-row
+// logsumexp; the backward recomputes the probabilities tile by tile from them
+// ("Walk through the FlashAttention algorithm ...", answer to "How does the
+// backward pass avoid storing the n x n attention matrix?"; "11.11 Flash
+// Attention", section "The Recomputation Trade-off").  The gradient formulas
+// are the chain rule of O = softmax(scale Q K^T) V (the pages give none):
+//   dV = P^T dO,  dP = dO V^T,  D = rowsum(dO o O),  dS = P o (dP - D),
+//   dQ = scale dS K,  dK = scale dS^T Q.
+//
+// Stage 1 (attn_bwd_preprocess_kernel): D and LSE*log2(e) per row into a
+//   padded workspace; zero the fp32 dQ accumulator.
+// Stage 2 (attn_bwd_kernel): one CTA per (batch, head, 128-key tile j).  It
+//   keeps K_j, V_j in shared memory and dK_j, dV_j in tensor memory, and walks
+//   the query tiles i (i >= j under the causal mask).  Per query tile:
+//     S^T = K_j Q_i^T            (tcgen05, TMEM)
+//     P^T = exp2(S^T c - LSE_i)  (registers -> TMEM as bf16, over S^T)
+//     dP^T = V_j dO_i^T          (tcgen05, TMEM)
+//     dV_j += P^T dO_i           (A operand read from TMEM)
+//     dS^T = P^T o (dP^T - D_i)  (registers -> shared memory as bf16)
+//     dK_j += dS^T Q_i ;  dQ_i-partial = dS K_j  (tcgen05)
+//   and adds the dQ partial into the fp32 accumulator with vector reductions.
+// Stage 3 (attn_bwd_dq_convert_kernel): dQ = bf16(scale * accumulator).
+#pragma once
+#include "ptx.cuh"
+
+namespace exattn {
+
+struct BwdParams {
+  CUtensorMap tm_q;  // 3-D {d, N, B*H}, box {64, 128, 1}, 128-byte swizzle
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
+  CUtensorMap tm_do;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  float* dq_acc;       // [BH, Np, d]
+  const float* dvec;   // [BH, Np]  D
+  const float* lse2;   // [BH, Np]  LSE * log2(e), +inf on padded rows
+  int N;
+  int Np;
+  int BH;
+  int ntiles;  // ceil(N / 128)
+  int causal;
+  float scale;
+  float scale_log2;
+  unsigned long long timeout_ns;
+};
+
+template <int D>
+struct BwdCfg {
+  // warps 0..3: compute, query columns 0..63; warps 4..7: columns 64..127;
+  // warps 8..11: dQ drain; warp 12: TMA producer; warp 13: MMA issuer.
+  static constexpr int kThreads = 448;
+  static constexpr uint32_t kTile = 128u * D * 2u;
+  static constexpr int kChunks = D / 64;
+  static constexpr uint32_t kOffK = 0;
+  static constexpr uint32_t kOffV = kTile;
+  static constexpr uint32_t kOffQ = 2 * kTile;   // 2 stages
+  static constexpr uint32_t kOffDO = 4 * kTile;  // 2 stages
+  static constexpr uint32_t kOffDS = 6 * kTile;  // 128 x 128 bf16
+  static constexpr uint32_t kOffVec = kOffDS + 32768;  // 2 stages x (LSE2[128], D[128]) fp32
+  static constexpr uint32_t kOffBar = kOffVec + 2048;
+  static constexpr uint32_t kSmem = kOffBar + 256;
+  // tensor-memory columns
+  static constexpr uint32_t kColDK = 0;
+  static constexpr uint32_t kColDV = D;
+  static constexpr uint32_t kColS = 2 * D;
+  static constexpr uint32_t kColDP = 2 * D + 128;
+  static constexpr uint32_t kColDQ = (D == 128) ? kColDP : 384;  // d=128: dQ reuses dP's columns
+};
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant__ BwdParams p) {
+  using C = BwdCfg<D>;
+  constexpr int kProducerWarp = 12;
+  constexpr int kMmaWarp = 13;
+  constexpr uint32_t TILE = C::kTile;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) record_status(kDevStatusBadSmemAlign, 200);
+    return;
+  }
+  uint8_t* sK = smem + C::kOffK;
+  uint8_t* sV = smem + C::kOffV;
+  uint8_t* sQ = smem + C::kOffQ;
+  uint8_t* sDO = smem + C::kOffDO;
+  uint8_t* sDS = smem + C::kOffDS;
+  float* sVec = reinterpret_cast<float*>(smem + C::kOffVec);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* bar_kv = bars + 0;
+  uint64_t* bar_qfull = bars + 1;   // [2]
+  uint64_t* bar_qempty = bars + 3;  // [2]
+  uint64_t* bar_s = bars + 5;       // S^T ready
+  uint64_t* bar_dp = bars + 6;      // dP^T ready
+  uint64_t* bar_p = bars + 7;       // P^T written (256 arrivals)
+  uint64_t* bar_ds = bars + 8;      // dS written to smem (256 arrivals)
+  uint64_t* bar_dsfree = bars + 9;  // dS smem consumed
+  uint64_t* bar_dqfull = bars + 10; // dQ partial ready in TMEM
+  uint64_t* bar_dqfree = bars + 11; // dQ partial read out (128 arrivals)
+  uint64_t* bar_final = bars + 12;  // all MMAs done
+  uint64_t* bar_drain = bars + 13;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int N = p.N;
+  const int T = p.ntiles;
+  // Key tile 0 first: under the causal mask it sees the most query tiles.
+  const int j = static_cast<int>(blockIdx.x) / p.BH;
+  const int bh = static_cast<int>(blockIdx.x) % p.BH;
+  const int i0 = p.causal ? j : 0;
+  const int n = T - i0;  // >= 1
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_kv, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar_qfull[s], 1);
+      mbar_init(&bar_qempty[s], 1);
+    }
+    mbar_init(bar_s, 1);
+    mbar_init(bar_dp, 1);
+    mbar_init(bar_p, 256);
+    mbar_init(bar_ds, 256);
+    mbar_init(bar_dsfree, 1);
+    mbar_init(bar_dqfull, 1);
+    mbar_init(bar_dqfree, 128);
+    mbar_init(bar_final, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint64_t tmo = p.timeout_ns;
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&p.tm_q);
+      prefetch_tensormap(&p.tm_k);
+      prefetch_tensormap(&p.tm_v);
+      prefetch_tensormap(&p.tm_do);
+      mbar_arrive_expect_tx(bar_kv, 2 * TILE);
+#pragma unroll
+      for (int c = 0; c < C::kChunks; ++c) {
+        tma_load_3d(sK + c * 16384, &p.tm_k, bar_kv, c * 64, j * 128, bh);
+        tma_load_3d(sV + c * 16384, &p.tm_v, bar_kv, c * 64, j * 128, bh);
+      }
+      int last_par0 = -1, last_par1 = -1;  // parity of the last load into each stage
+      bool ok = true;
+      for (int it = 0; it < n; ++it) {
+        const int st = it & 1;
+        const uint32_t ph = (it >> 1) & 1;
+        if (!mbar_wait(&bar_qempty[st], ph ^ 1u, abort_flag, tmo, 201)) {
+          ok = false;
+          break;
+        }
+        const int i = i0 + it;
+        mbar_arrive_expect_tx(&bar_qfull[st], 2 * TILE + 1024);
+#pragma unroll
+        for (int c = 0; c < C::kChunks; ++c) {
+          tma_load_3d(sQ + st * TILE + c * 16384, &p.tm_q, &bar_qfull[st], c * 64, i * 128, bh);
+          tma_load_3d(sDO + st * TILE + c * 16384, &p.tm_do, &bar_qfull[st], c * 64, i * 128, bh);
+        }
+        const size_t vrow = static_cast<size_t>(bh) * p.Np + static_cast<size_t>(i) * 128;
+        bulk_load(sVec + st * 256, p.lse2 + vrow, 512, &bar_qfull[st]);
+        bulk_load(sVec + st * 256 + 128, p.dvec + vrow, 512, &bar_qfull[st]);
+        if (st == 0) last_par0 = static_cast<int>(ph); else last_par1 = static_cast<int>(ph);
+      }
+      if (!ok) {
+        drain_wait(bar_kv, 0, 202);
+        if (last_par0 >= 0) drain_wait(&bar_qfull[0], static_cast<uint32_t>(last_par0), 203);
+        if (last_par1 >= 0) drain_wait(&bar_qfull[1], static_cast<uint32_t>(last_par1), 203);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_t = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T: both operands K-major
+      constexpr uint32_t idesc_kv = idesc_bf16_f32(128, D, 0, 1);   // dV, dK: B = dO / Q MN-major
+      constexpr uint32_t idesc_q = idesc_bf16_f32(128, D, 1, 1);    // dQ: A = dS MN-major, B = K MN-major
+      const uint32_t sK0 = smem_u32(sK), sV0 = smem_u32(sV), sQ0 = smem_u32(sQ), sDO0 = smem_u32(sDO);
+      const uint32_t sDS0 = smem_u32(sDS);
+      // X[128 x 128] = A[128 x D] B[128 x D]^T, both K-major D-wide tiles
+      auto issue_t = [&](uint32_t dcol, uint32_t a0, uint32_t b0) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ss(tmem + dcol, smem_desc_sw128(a0 + off, 16, 1024), smem_desc_sw128(b0 + off, 16, 1024), idesc_t,
+                 kk > 0 ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(bar_kv, 0, abort_flag, tmo, 210) && mbar_wait(&bar_qfull[0], 0, abort_flag, tmo, 211);
+      if (ok) {
+        tc_fence_after();
+        issue_t(C::kColS, sK0, sQ0);
+        tc_commit(bar_s);
+        issue_t(C::kColDP, sV0, sDO0);
+        tc_commit(bar_dp);
+      }
+      for (int it = 0; it < n && ok; ++it) {
+        const int st = it & 1;
+        // dV += P^T dO_i   (A = P^T from TMEM, K = 128 queries; queries 0..63
+        // sit in columns [0,32) of the score block, 64..127 in [64,96))
+        if (!mbar_wait(bar_p, it & 1, abort_flag, tmo, 212)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + C::kColDV, tmem + C::kColS + (kk >> 2) * 64 + (kk & 3) * 8,
+                 smem_desc_sw128(sDO0 + st * TILE + kk * 2048, 16384, 1024), idesc_kv,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+        // next S^T as early as possible: the softmax of tile it+1 overlaps dK, dQ of tile it
+        if (it + 1 < n) {
+          const int st1 = (it + 1) & 1;
+          if (!mbar_wait(&bar_qfull[st1], ((it + 1) >> 1) & 1, abort_flag, tmo, 213)) break;
+          tc_fence_after();
+          issue_t(C::kColS, sK0, sQ0 + st1 * TILE);
+          tc_commit(bar_s);
+        }
+        if (!mbar_wait(bar_ds, it & 1, abort_flag, tmo, 214)) break;
+        tc_fence_after();
+        // dK += dS^T Q_i   (A = dS^T K-major in smem, B = Q_i MN-major)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t offa = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ss(tmem + C::kColDK, smem_desc_sw128(sDS0 + offa, 16, 1024),
+                 smem_desc_sw128(sQ0 + st * TILE + kk * 2048, 16384, 1024), idesc_kv,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+        }
+        if (D != 128 && it > 0) {  // separate dQ columns: only the previous dQ must be drained
+          if (!mbar_wait(bar_dqfree, (it - 1) & 1, abort_flag, tmo, 215)) break;
+          tc_fence_after();
+        }
+        // dQ_i partial = dS K_j   (A = dS MN-major in smem, B = K_j MN-major)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + C::kColDQ, smem_desc_sw128(sDS0 + kk * 2048, 16384, 1024),
+                 smem_desc_sw128(sK0 + kk * 2048, 16384, 1024), idesc_q, kk > 0 ? 1u : 0u);
+        tc_commit(bar_dqfull);
+        tc_commit(&bar_qempty[st]);
+        tc_commit(bar_dsfree);
+        if (it + 1 < n) {
+          if (D == 128) {  // dP^T(it+1) overwrites the dQ partial: wait until it is read out
+            if (!mbar_wait(bar_dqfree, it & 1, abort_flag, tmo, 216)) break;
+            tc_fence_after();
+          }
+          issue_t(C::kColDP, sV0, sDO0 + ((it + 1) & 1) * TILE);
+          tc_commit(bar_dp);
+        }
+      }
+      tc_commit(bar_final);
+      tc_commit(bar_drain);
+      drain_wait(bar_drain, 0, 217);
+    }
+    __syncwarp();
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ compute
+    const int h = warp >> 2;  // query-column half
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;  // key row in the tile
+    const int key = j * 128 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    // Each half reads its 64 score columns and writes its 64 bf16 probabilities
+    // (32 columns) over the first half of those same columns, so the two
+    // halves never touch each other's columns.
+    const uint32_t tS = tmem + lane_off + C::kColS + 64 * h;
+    const uint32_t tP = tS;
+    const uint32_t tDP = tmem + lane_off + C::kColDP + 64 * h;
+    const float c = p.scale_log2;
+    const bool key_ok = key < N;
+    uint8_t* ds_row = sDS + h * 16384 + r * 128;
+    bool ok = true;
+    for (int it = 0; it < n; ++it) {
+      const int st = it & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_s, it & 1, abort_flag, tmo, 220))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[64];
+      tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_wait_ld();
+      const float* lse2 = sVec + st * 256 + 64 * h;
+      const float* dv = sVec + st * 256 + 128 + 64 * h;
+      const bool diag = p.causal && (it == 0);
+      float pf[64];
+#pragma unroll
+      for (int e = 0; e < 64; ++e) {
+        float pv = ex2(fmaf(__uint_as_float(sr[e]), c, -lse2[e]));
+        if (!key_ok || (diag && r > 64 * h + e)) pv = 0.f;
+        pf[e] = pv;
+      }
+      uint32_t pk[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(pf[2 * e], pf[2 * e + 1]);
+      tmem_st16(tP, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
+      tmem_st16(tP + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_p);
+
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_dp, it & 1, abort_flag, tmo, 221))) {
+        ok = false;
+        break;
+      }
+      if (it > 0 && !__all_sync(0xffffffffu, mbar_wait(bar_dsfree, (it - 1) & 1, abort_flag, tmo, 222))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        uint32_t dpr[32];
+        tmem_ld32(tDP + 32 * ch, dpr);
+        tmem_wait_ld();
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int e0 = 32 * ch + 2 * e;
+          const float d0 = pf[e0] * (__uint_as_float(dpr[2 * e]) - dv[e0]);
+          const float d1 = pf[e0 + 1] * (__uint_as_float(dpr[2 * e + 1]) - dv[e0 + 1]);
+          w[e] = pack_bf16x2(d0, d1);
+        }
+        // 128-byte swizzle: 16-byte unit u of row r lives at unit (u ^ (r & 7))
+#pragma unroll
+        for (int u4 = 0; u4 < 4; ++u4) {
+          const int u = 4 * ch + u4;
+          *reinterpret_cast<uint4*>(ds_row + ((u ^ (r & 7)) << 4)) =
+              make_uint4(w[4 * u4], w[4 * u4 + 1], w[4 * u4 + 2], w[4 * u4 + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar_ds);
+    }
+    // epilogue: half 0 writes dK (times scale), half 1 writes dV
+    if (ok && __all_sync(0xffffffffu, mbar_wait(bar_final, 0, abort_flag, tmo, 223))) {
+      tc_fence_after();
+      const uint32_t tAcc = tmem + lane_off + (h == 0 ? C::kColDK : C::kColDV);
+      const float mul = (h == 0) ? p.scale : 1.0f;
+      __nv_bfloat16* out = (h == 0 ? p.dk : p.dv) + (static_cast<size_t>(bh) * N + key) * D;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t a[32];
+        tmem_ld32(tAcc + 32 * cc, a);
+        tmem_wait_ld();
+        if (key_ok) {
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            w[e] = pack_bf16x2(__uint_as_float(a[2 * e]) * mul, __uint_as_float(a[2 * e + 1]) * mul);
+          uint4* dst = reinterpret_cast<uint4*>(out + 32 * cc);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+        }
+      }
+    }
+  } else if (warp < 12) {
+    // ------------------------------------------------------------ dQ drain
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;  // query row in the tile
+    const uint32_t tQ = tmem + (static_cast<uint32_t>(wq * 32) << 16) + C::kColDQ;
+    for (int it = 0; it < n; ++it) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_dqfull, it & 1, abort_flag, tmo, 230))) break;
+      tc_fence_after();
+      float* dst = p.dq_acc + (static_cast<size_t>(bh) * p.Np + static_cast<size_t>(i0 + it) * 128 + r) * D;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t a[32];
+        tmem_ld32(tQ + 32 * cc, a);
+        tmem_wait_ld();
+        if (cc == D / 32 - 1) {  // every read of this partial is complete: hand the columns back
+          tc_fence_before();
+          mbar_arrive(bar_dqfree);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          red_add_v4(dst + 32 * cc + 4 * e, __uint_as_float(a[4 * e]), __uint_as_float(a[4 * e + 1]),
+                     __uint_as_float(a[4 * e + 2]), __uint_as_float(a[4 * e + 3]));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------- stage 1
+// One row per (d/8) lanes; each lane reads 8 elements (16 bytes) of O and dO.
+template <int D>
+__global__ void __launch_bounds__(256) attn_bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o,
+                                                                  const __nv_bfloat16* __restrict__ dO,
+                                                                  const float* __restrict__ lse,
+                                                                  float* __restrict__ dvec,
+                                                                  float* __restrict__ lse2,
+                                                                  float* __restrict__ dq_acc, int BH, int N,
+                                                                  int Np) {
+  constexpr int LPR = D / 8;            // lanes per row
+  constexpr int RPB = 256 / LPR;        // rows per block
+  const int sub = threadIdx.x % LPR;
+  const long long row = static_cast<long long>(blockIdx.x) * RPB + threadIdx.x / LPR;  // over BH * Np
+  const long long total = static_cast<long long>(BH) * Np;
+  float acc = 0.f;
+  const bool in = row < total;
+  const int bh = in ? static_cast<int>(row / Np) : 0;
+  const int i = in ? static_cast<int>(row % Np) : 0;
+  const bool valid = in && i < N;
+  if (valid) {
+    const size_t off = (static_cast<size_t>(bh) * N + i) * D + sub * 8;
+    const uint4 a = *reinterpret_cast<const uint4*>(o + off);
+    const uint4 b = *reinterpret_cast<const uint4*>(dO + off);
+    const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 x = __bfloat1622float2(pa[e]);
+      const float2 y = __bfloat1622float2(pb[e]);
+      acc = fmaf(x.x, y.x, acc);
+      acc = fmaf(x.y, y.y, acc);
+    }
+  }
+#pragma unroll
+  for (int m = LPR / 2; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+  if (in) {
+    float4* z = reinterpret_cast<float4*>(dq_acc + static_cast<size_t>(row) * D + sub * 8);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (sub == 0) {
+      dvec[row] = valid ? acc : 0.f;
+      lse2[row] = valid ? lse[static_cast<size_t>(bh) * N + i] * 1.4426950408889634f : INFINITY;
+    }
+  }
+}
+
+inline void launch_bwd_preprocess(const __nv_bfloat16* o, const __nv_bfloat16* dO, const float* lse, float* dvec,
+                                  float* lse2, float* dq_acc, int BH, int N, int Np, int d, cudaStream_t s) {
+  const long long rows = static_cast<long long>(BH) * Np;
+  if (d == 64) {
+    const unsigned blocks = static_cast<unsigned>((rows + 31) / 32);
+    attn_bwd_preprocess_kernel<64><<<blocks, 256, 0, s>>>(o, dO, lse, dvec, lse2, dq_acc, BH, N, Np);
+  } else {
+    const unsigned blocks = static_cast<unsigned>((rows + 15) / 16);
+    attn_bwd_preprocess_kernel<128><<<blocks, 256, 0, s>>>(o, dO, lse, dvec, lse2, dq_acc, BH, N, Np);
+  }
+}
+
+// ---------------------------------------------------------------- stage 3
+// Each thread converts 8 consecutive elements of one row.
+__global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float* __restrict__ dq_acc,
+                                                                  __nv_bfloat16* __restrict__ dq, int N, int Np,
+                                                                  int d, float scale, long long total8) {
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= total8) return;
+  const long long e = t * 8;                    // element index in [BH, N, d]
+  const long long rowN = e / d;                 // bh * N + i
+  const int col = static_cast<int>(e - rowN * d);
+  const long long bh = rowN / N;
+  const long long i = rowN - bh * N;
+  const float4* src = reinterpret_cast<const float4*>(dq_acc + (bh * Np + i) * d + col);
+  const float4 a = src[0], b = src[1];
+  uint4 w;
+  w.x = pack_bf16x2(a.x * scale, a.y * scale);
+  w.y = pack_bf16x2(a.z * scale, a.w * scale);
+  w.z = pack_bf16x2(b.x * scale, b.y * scale);
+  w.w = pack_bf16x2(b.z * scale, b.w * scale);
+  *reinterpret_cast<uint4*>(dq + e) = w;
+}
+
+inline void launch_bwd_dq_convert(const float* dq_acc, __nv_bfloat16* dq, int BH, int N, int Np, int d, float scale,
+                                  cudaStream_t s) {
+  const long long total8 = static_cast<long long>(BH) * N * d / 8;
+  const unsigned blocks = static_cast<unsigned>((total8 + 255) / 256);
+  attn_bwd_dq_convert_kernel<<<blocks, 256, 0, s>>>(dq_acc, dq, N, Np, d, scale, total8);
+}
+
+}  // namespace exattn

@@ -1,0 +1,293 @@
+// C ABI of exattn: argument checks, TMA tensor maps and kernel launches.
+// The operations themselves are documented in include/exattn.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "exattn.h"
+#include "ptx.cuh"
+#include "fwd.cuh"
+#include "bwd.cuh"
+
+namespace {
+
+using exattn::BwdParams;
+using exattn::FwdParams;
+
+constexpr unsigned long long kDefaultTimeoutNs = 1000000000ull;  // 1 s per wait
+constexpr int kMaxDevices = 64;
+
+// ------------------------------------------------------------------ checks
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 0 = proceed, 1 = empty problem (nothing to do), -1 = invalid
+int check_sizes(int B, int H, int N, int d) {
+  if (B < 0 || H < 0 || N < 0) return -1;
+  if (d != 64 && d != 128) return -1;
+  if (B == 0 || H == 0 || N == 0) return 1;
+  const long long bh = static_cast<long long>(B) * H;
+  if (bh > 0x7fffffffLL) return -1;
+  const long long nblk = (static_cast<long long>(N) + 255) / 256;
+  if (nblk * bh > 0x7fffffffLL) return -1;  // grid size
+  return 0;
+}
+
+bool check_scale(float scale) { return std::isfinite(scale) && scale > 0.f; }
+
+size_t padded_rows(int N) { return (static_cast<size_t>(N) + 127) / 128 * 128; }
+
+struct Workspace {
+  float* dq_acc;  // [BH, Np, d]
+  float* dvec;    // [BH, Np]
+  float* lse2;    // [BH, Np]
+};
+
+size_t workspace_bytes(int B, int H, int N, int d) {
+  const size_t bh = static_cast<size_t>(B) * H;
+  const size_t np = padded_rows(N);
+  return bh * np * d * 4 + 2 * bh * np * 4;
+}
+
+Workspace carve(void* ws, int B, int H, int N, int d) {
+  const size_t bh = static_cast<size_t>(B) * H;
+  const size_t np = padded_rows(N);
+  float* base = static_cast<float*>(ws);
+  return Workspace{base, base + bh * np * d, base + bh * np * d + bh * np};
+}
+
+// ------------------------------------------------------------------ device
+int check_device(int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_LAUNCH;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return ATTN_ERR_LAUNCH;
+  if (major != 10 || minor != 0) return ATTN_ERR_UNSUPPORTED_DEVICE;
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED_DEVICE;
+  *dev_out = dev;
+  return ATTN_OK;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(ptr);
+  }();
+  return fn;
+}
+
+// 3-D view {d, N, B*H} of a contiguous bf16 [B,H,N,d] tensor; box {64, 128, 1}
+// with 128-byte swizzle.  Rows past N of a head read as zeros.
+bool make_map_bf16(CUtensorMap* m, const void* base, int BH, int N, int d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Per-device, per-kernel one-time opt-in to large dynamic shared memory.
+template <typename K>
+bool ensure_smem_attr(K kernel, int dev, std::atomic<int>* flags, int bytes) {
+  if (flags[dev].load(std::memory_order_acquire)) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return false;
+  flags[dev].store(1, std::memory_order_release);
+  return true;
+}
+
+std::atomic<int> g_fwd64_attr[kMaxDevices];
+std::atomic<int> g_fwd128_attr[kMaxDevices];
+std::atomic<int> g_bwd64_attr[kMaxDevices];
+std::atomic<int> g_bwd128_attr[kMaxDevices];
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH; }
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+             float scale, int causal, attn_stream_t stream) {
+  const int sz = check_sizes(B, H, N, d);
+  if (sz < 0 || !check_scale(scale)) return ATTN_ERR_INVALID;
+  if (sz == 1) return ATTN_OK;
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return ATTN_ERR_INVALID;
+  int dev = 0;
+  if (int st = check_device(&dev)) return st;
+
+  FwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  const int BH = B * H;
+  if (!make_map_bf16(&p.tm_q, q, BH, N, d) || !make_map_bf16(&p.tm_k, k, BH, N, d) ||
+      !make_map_bf16(&p.tm_v, v, BH, N, d))
+    return ATTN_ERR_LAUNCH;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.N = N;
+  p.BH = BH;
+  p.nblocks = (N + 255) / 256;
+  p.causal = causal ? 1 : 0;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = kDefaultTimeoutNs;
+  const dim3 grid(static_cast<unsigned>(p.nblocks) * static_cast<unsigned>(BH));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64) {
+    constexpr int smem = exattn::FwdCfg<64>::kSmem;
+    if (!ensure_smem_attr(exattn::attn_fwd_kernel<64>, dev, g_fwd64_attr, smem)) return ATTN_ERR_LAUNCH;
+    exattn::attn_fwd_kernel<64><<<grid, exattn::FwdCfg<64>::kThreads, smem, s>>>(p);
+  } else {
+    constexpr int smem = exattn::FwdCfg<128>::kSmem;
+    if (!ensure_smem_attr(exattn::attn_fwd_kernel<128>, dev, g_fwd128_attr, smem)) return ATTN_ERR_LAUNCH;
+    exattn::attn_fwd_kernel<128><<<grid, exattn::FwdCfg<128>::kThreads, smem, s>>>(p);
+  }
+  return launch_status();
+}
+
+size_t attn_bwd_workspace_bytes(int B, int H, int N, int d) {
+  if (check_sizes(B, H, N, d) != 0) return 0;
+  return workspace_bytes(B, H, N, d);
+}
+
+int attn_bwd_preprocess(const void* o, const void* dO, const float* lse, int B, int H, int N, int d,
+                        void* workspace, size_t workspace_bytes_given, attn_stream_t stream) {
+  const int sz = check_sizes(B, H, N, d);
+  if (sz < 0) return ATTN_ERR_INVALID;
+  if (sz == 1) return ATTN_OK;
+  if (!o || !dO || !lse || !workspace) return ATTN_ERR_INVALID;
+  if (!aligned16(o) || !aligned16(dO) || !aligned16(lse) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return ATTN_ERR_INVALID;
+  if (workspace_bytes_given < workspace_bytes(B, H, N, d)) return ATTN_ERR_INVALID;
+  int dev = 0;
+  if (int st = check_device(&dev)) return st;
+  const Workspace ws = carve(workspace, B, H, N, d);
+  const int BH = B * H;
+  const int np = static_cast<int>(padded_rows(N));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  exattn::launch_bwd_preprocess(static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse,
+                                ws.dvec, ws.lse2, ws.dq_acc, BH, N, np, d, s);
+  return launch_status();
+}
+
+int attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, int B, int H,
+                  int N, int d, float scale, int causal, void* workspace, size_t workspace_bytes_given,
+                  attn_stream_t stream) {
+  const int sz = check_sizes(B, H, N, d);
+  if (sz < 0 || !check_scale(scale)) return ATTN_ERR_INVALID;
+  if (sz == 1) return ATTN_OK;
+  if (!q || !k || !v || !dO || !dk || !dv || !workspace) return ATTN_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return ATTN_ERR_INVALID;
+  if (workspace_bytes_given < workspace_bytes(B, H, N, d)) return ATTN_ERR_INVALID;
+  int dev = 0;
+  if (int st = check_device(&dev)) return st;
+  const Workspace ws = carve(workspace, B, H, N, d);
+  BwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  const int BH = B * H;
+  if (!make_map_bf16(&p.tm_q, q, BH, N, d) || !make_map_bf16(&p.tm_k, k, BH, N, d) ||
+      !make_map_bf16(&p.tm_v, v, BH, N, d) || !make_map_bf16(&p.tm_do, dO, BH, N, d))
+    return ATTN_ERR_LAUNCH;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.dq_acc = ws.dq_acc;
+  p.dvec = ws.dvec;
+  p.lse2 = ws.lse2;
+  p.N = N;
+  p.Np = static_cast<int>(padded_rows(N));
+  p.BH = BH;
+  p.ntiles = (N + 127) / 128;
+  p.causal = causal ? 1 : 0;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = kDefaultTimeoutNs;
+  const dim3 grid(static_cast<unsigned>(p.ntiles) * static_cast<unsigned>(BH));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64) {
+    constexpr int smem = exattn::BwdCfg<64>::kSmem;
+    if (!ensure_smem_attr(exattn::attn_bwd_kernel<64>, dev, g_bwd64_attr, smem)) return ATTN_ERR_LAUNCH;
+    exattn::attn_bwd_kernel<64><<<grid, exattn::BwdCfg<64>::kThreads, smem, s>>>(p);
+  } else {
+    constexpr int smem = exattn::BwdCfg<128>::kSmem;
+    if (!ensure_smem_attr(exattn::attn_bwd_kernel<128>, dev, g_bwd128_attr, smem)) return ATTN_ERR_LAUNCH;
+    exattn::attn_bwd_kernel<128><<<grid, exattn::BwdCfg<128>::kThreads, smem, s>>>(p);
+  }
+  return launch_status();
+}
+
+int attn_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, const void* workspace,
+                        size_t workspace_bytes_given, attn_stream_t stream) {
+  const int sz = check_sizes(B, H, N, d);
+  if (sz < 0 || !check_scale(scale)) return ATTN_ERR_INVALID;
+  if (sz == 1) return ATTN_OK;
+  if (!dq || !workspace) return ATTN_ERR_INVALID;
+  if (!aligned16(dq) || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return ATTN_ERR_INVALID;
+  if (workspace_bytes_given < workspace_bytes(B, H, N, d)) return ATTN_ERR_INVALID;
+  int dev = 0;
+  if (int st = check_device(&dev)) return st;
+  const Workspace ws = carve(const_cast<void*>(workspace), B, H, N, d);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  exattn::launch_bwd_dq_convert(ws.dq_acc, static_cast<__nv_bfloat16*>(dq), B * H, N,
+                                static_cast<int>(padded_rows(N)), d, scale, s);
+  return launch_status();
+}
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+             void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, void* workspace,
+             size_t workspace_bytes_given, attn_stream_t stream) {
+  const int sz = check_sizes(B, H, N, d);
+  if (sz < 0 || !check_scale(scale)) return ATTN_ERR_INVALID;
+  if (sz == 1) return ATTN_OK;
+  if (!dq) return ATTN_ERR_INVALID;
+  int st = attn_bwd_preprocess(o, dO, lse, B, H, N, d, workspace, workspace_bytes_given, stream);
+  if (st) return st;
+  st = attn_bwd_dkdv(q, k, v, dO, dk, dv, B, H, N, d, scale, causal, workspace, workspace_bytes_given, stream);
+  if (st) return st;
+  return attn_bwd_dq_convert(dq, B, H, N, d, scale, workspace, workspace_bytes_given, stream);
+}
+
+int attn_get_device_status(attn_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_LAUNCH;
+  unsigned int word = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&word, exattn::g_status_word, sizeof(word)) != cudaSuccess) return ATTN_ERR_LAUNCH;
+  if (word == 0) return ATTN_OK;
+  if (cudaMemcpyToSymbol(exattn::g_status_word, &zero, sizeof(zero)) != cudaSuccess ||
+      cudaMemcpyToSymbol(exattn::g_status_site, &zero, sizeof(zero)) != cudaSuccess)
+    return ATTN_ERR_LAUNCH;
+  return (word & exattn::kDevStatusTimeout) ? ATTN_ERR_TIMEOUT : ATTN_ERR_LAUNCH;
+}
+
+const char* attn_status_string(int status) {
+  switch (status) {
+    case ATTN_OK: return "ATTN_OK";
+    case ATTN_ERR_INVALID: return "ATTN_ERR_INVALID";
+    case ATTN_ERR_UNSUPPORTED_DEVICE: return "ATTN_ERR_UNSUPPORTED_DEVICE";
+    case ATTN_ERR_LAUNCH: return "ATTN_ERR_LAUNCH";
+    case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT";
+    default: return "ATTN_ERR_UNKNOWN";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,347 @@
+// Forward kernel: O = softmax(scale Q K^T) V and LSE, tile by tile with an
+// online softmax ("11.11 Flash Attention", sections "Flash Attention: The Key
+// Insight" and "The Tiling Algorithm"; loop order of section "Flash
+// Attention 2": Q blocks outside, K/V blocks inside, parallel over batch x
+// heads x Q blocks).
+//
+// One CTA owns a 256-row block of queries of one (batch, head), split into two
+// 128-row sub-tiles that ping-pong on the tensor core (while the softmax of
+// one sub-tile runs, the MMAs of the other do).  Roles (320 threads):
+//   warps 0..3    softmax of sub-tile 0 (one thread per query row)
+//   warps 4..7    softmax of sub-tile 1
+//   warp 8        TMA producer: Q (once), then K_j and V_j into a smem ring
+//   warp 9        TMEM allocator; lane 0 issues every tcgen05.mma
+// Tensor memory (512 columns x 128 lanes of 32 bit), per sub-tile k:
+//   columns [256k, 256k+128)      S_k = Q_k K_j^T (fp32); P_k (bf16 pairs) is
+//                                 written back over its first 64 columns
+//   columns [256k+128, +d)        O_k accumulator (fp32)
+// The softmax keeps, per row, a reference maximum and the running sum l;
+// the division by l happens once at the end (section "Flash Attention 2":
+// fewer non-matmul operations).  The reference maximum only moves when a
+// tile's maximum exceeds it by more than 2^8 in probability units, so O is
+// rescaled in TMEM rarely; this is exact, because O and l always share the
+// same reference.
+#pragma once
+#include "ptx.cuh"
+
+namespace exattn {
+
+struct FwdParams {
+  CUtensorMap tm_q;  // 3-D {d, N, B*H}, box {64, 128, 1}, 128-byte swizzle
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
+  __nv_bfloat16* o;
+  float* lse;
+  int N;
+  int BH;
+  int nblocks;  // ceil(N / 256)
+  int causal;
+  float scale;       // softmax scale
+  float scale_log2;  // scale * log2(e)
+  unsigned long long timeout_ns;
+};
+
+template <int D>
+struct FwdCfg {
+  static constexpr int kThreads = 320;
+  static constexpr uint32_t kTile = 128u * D * 2u;  // one 128-row bf16 tile
+  static constexpr int kSlots = (D == 128) ? 4 : 8;  // K/V ring slots
+  static constexpr int kChunks = D / 64;             // 64-column swizzle chunks per tile
+  static constexpr uint32_t kBarOff = (2 + kSlots) * kTile;
+  static constexpr uint32_t kSmem = kBarOff + 256;
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1) attn_fwd_kernel(const __grid_constant__ FwdParams p) {
+  using C = FwdCfg<D>;
+  constexpr int kProducerWarp = 8;
+  constexpr int kMmaWarp = 9;
+  constexpr int SLOTS = C::kSlots;
+  constexpr uint32_t TILE = C::kTile;
+  extern __shared__ __align__(1024) uint8_t smem[];
+
+  if (smem_u32(smem) & 1023u) {  // 128-byte swizzle needs 1024-byte aligned tiles
+    if (threadIdx.x == 0) record_status(kDevStatusBadSmemAlign, 100);
+    return;
+  }
+  uint8_t* sQ = smem;
+  uint8_t* sKV = smem + 2 * TILE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* bar_q = bars;
+  uint64_t* bar_full = bars + 1;
+  uint64_t* bar_empty = bars + 1 + SLOTS;
+  uint64_t* bar_s = bars + 1 + 2 * SLOTS;  // [2] S_k ready
+  uint64_t* bar_p = bar_s + 2;             // [2] P_k written (and O_k corrected)
+  uint64_t* bar_o = bar_p + 2;             // [2] last P_k V done
+  uint64_t* bar_drain = bar_o + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int N = p.N;
+  const int T = (N + 127) >> 7;
+  // Heaviest query blocks first (they see the most keys under the causal mask).
+  const int qb = p.nblocks - 1 - static_cast<int>(blockIdx.x) / p.BH;
+  const int bh = static_cast<int>(blockIdx.x) % p.BH;
+  int n_sub[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int row0 = qb * 256 + k * 128;
+    n_sub[k] = (row0 >= N) ? 0 : (p.causal ? min(T, 2 * qb + k + 1) : T);
+  }
+  const int nmax = max(n_sub[0], n_sub[1]);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < SLOTS; ++s) {
+      mbar_init(&bar_full[s], 1);
+      mbar_init(&bar_empty[s], 1);
+    }
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(&bar_s[k], 1);
+      mbar_init(&bar_p[k], 128);
+      mbar_init(&bar_o[k], 1);
+    }
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint64_t tmo = p.timeout_ns;
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && nmax > 0) {
+      prefetch_tensormap(&p.tm_q);
+      prefetch_tensormap(&p.tm_k);
+      prefetch_tensormap(&p.tm_v);
+      mbar_arrive_expect_tx(bar_q, TILE * (n_sub[1] > 0 ? 2u : 1u));
+#pragma unroll
+      for (int c = 0; c < C::kChunks; ++c) {
+        tma_load_3d(sQ + c * 16384, &p.tm_q, bar_q, c * 64, qb * 256, bh);
+        if (n_sub[1] > 0) tma_load_3d(sQ + TILE + c * 16384, &p.tm_q, bar_q, c * 64, qb * 256 + 128, bh);
+      }
+      int last_par[SLOTS];
+#pragma unroll
+      for (int s = 0; s < SLOTS; ++s) last_par[s] = -1;
+      bool ok = true;
+      for (int j = 0; j < nmax && ok; ++j) {
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          const int idx = 2 * j + x;
+          const int slot = idx % SLOTS;
+          const uint32_t ph = (idx / SLOTS) & 1;
+          if (!mbar_wait(&bar_empty[slot], ph ^ 1u, abort_flag, tmo, 101)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar_full[slot], TILE);
+          const CUtensorMap* m = x ? &p.tm_v : &p.tm_k;
+#pragma unroll
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_3d(sKV + slot * TILE + c * 16384, m, &bar_full[slot], c * 64, j * 128, bh);
+#pragma unroll
+          for (int s = 0; s < SLOTS; ++s)
+            if (s == slot) last_par[s] = static_cast<int>(ph);
+        }
+      }
+      if (!ok) {  // error path: let the copies already in flight land
+        drain_wait(bar_q, 0, 102);
+#pragma unroll
+        for (int s = 0; s < SLOTS; ++s)
+          if (last_par[s] >= 0) drain_wait(&bar_full[s], static_cast<uint32_t>(last_par[s]), 103);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && nmax > 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);  // Q, K both K-major
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);    // P from TMEM, V MN-major
+      const uint32_t sq0 = smem_u32(sQ);
+      const uint32_t skv0 = smem_u32(sKV);
+      auto kslot = [&](int j) { return (2 * j) % SLOTS; };
+      auto kph = [&](int j) { return static_cast<uint32_t>(((2 * j) / SLOTS) & 1); };
+      auto vslot = [&](int j) { return (2 * j + 1) % SLOTS; };
+      auto vph = [&](int j) { return static_cast<uint32_t>(((2 * j + 1) / SLOTS) & 1); };
+      auto issue_s = [&](int k, int slot) {
+        const uint32_t a0 = sq0 + k * TILE, b0 = skv0 + slot * TILE;
+        const uint32_t dt = tmem + k * 256;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ss(dt, smem_desc_sw128(a0 + off, 16, 1024), smem_desc_sw128(b0 + off, 16, 1024), idesc_s,
+                 kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int k, int slot, bool acc) {
+        const uint32_t b0 = skv0 + slot * TILE;
+        const uint32_t dt = tmem + k * 256 + 128;
+        const uint32_t at = tmem + k * 256;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          mma_ts(dt, at + kk * 8, smem_desc_sw128(b0 + kk * 2048, 16384, 1024), idesc_o,
+                 (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      const int n0 = n_sub[0], n1 = n_sub[1];
+      bool ok = mbar_wait(bar_q, 0, abort_flag, tmo, 110);
+      ok = ok && mbar_wait(&bar_full[kslot(0)], kph(0), abort_flag, tmo, 111);
+      if (ok) {
+        tc_fence_after();
+        if (n0 > 0) {
+          issue_s(0, kslot(0));
+          tc_commit(&bar_s[0]);
+        }
+        if (n1 > 0) {
+          issue_s(1, kslot(0));
+          tc_commit(&bar_s[1]);
+        }
+        tc_commit(&bar_empty[kslot(0)]);
+      }
+      for (int j = 0; j < nmax && ok; ++j) {
+        const bool knext = (j + 1 < nmax);
+        if (!mbar_wait(&bar_full[vslot(j)], vph(j), abort_flag, tmo, 112)) break;
+        tc_fence_after();
+        if (j < n0) {
+          if (!mbar_wait(&bar_p[0], j & 1, abort_flag, tmo, 113)) break;
+          tc_fence_after();
+          issue_pv(0, vslot(j), j > 0);
+          if (j == n0 - 1) tc_commit(&bar_o[0]);
+        }
+        if (knext) {
+          if (!mbar_wait(&bar_full[kslot(j + 1)], kph(j + 1), abort_flag, tmo, 114)) break;
+          tc_fence_after();
+        }
+        if (j + 1 < n0) {
+          issue_s(0, kslot(j + 1));
+          tc_commit(&bar_s[0]);
+        }
+        if (j < n1) {
+          if (!mbar_wait(&bar_p[1], j & 1, abort_flag, tmo, 115)) break;
+          tc_fence_after();
+          issue_pv(1, vslot(j), j > 0);
+          if (j == n1 - 1) tc_commit(&bar_o[1]);
+        }
+        tc_commit(&bar_empty[vslot(j)]);
+        if (j + 1 < n1) {
+          issue_s(1, kslot(j + 1));
+          tc_commit(&bar_s[1]);
+        }
+        if (knext) tc_commit(&bar_empty[kslot(j + 1)]);
+      }
+      // All MMAs issued by this thread must be complete before TMEM is freed.
+      tc_commit(bar_drain);
+      drain_wait(bar_drain, 0, 116);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int k = warp >> 2;        // sub-tile
+    const int wq = warp & 3;        // TMEM lane quadrant
+    const int row = wq * 32 + lane;
+    const int q_row = qb * 256 + k * 128 + row;
+    const uint32_t tS = tmem + (static_cast<uint32_t>(wq * 32) << 16) + k * 256;
+    const uint32_t tO = tS + 128;
+    const int n = k ? n_sub[1] : n_sub[0];
+    const float c = p.scale_log2;
+    const float thr = 8.0f / c;  // reference max moves only if exps would exceed 2^8
+    float m_ref = -INFINITY;
+    float l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      // warp-uniform outcome: the tcgen05.ld/st below are warp-collective
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar_s[k], j & 1, abort_flag, tmo, 120 + k))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[128];
+      tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+      tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+      tmem_wait_ld();
+      float s[128];
+#pragma unroll
+      for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(sr[i]);
+      const int key0 = j * 128;
+      const bool diag = p.causal && (j == 2 * qb + k);
+      if (diag || key0 + 128 > N) {
+        const int lim = min(diag ? row : 127, N - 1 - key0);  // last visible column
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (i > lim) s[i] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+      const float m_new = (mx > m_ref + thr) ? mx : m_ref;
+      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+      const float alpha = ex2((m_ref - m_use) * c);
+      const float neg = -m_use * c;
+      float sum = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        const float p0 = ex2(fmaf(s[2 * i], c, neg));
+        const float p1 = ex2(fmaf(s[2 * i + 1], c, neg));
+        sum += p0 + p1;
+        pk[i] = pack_bf16x2(p0, p1);
+      }
+      l = l * alpha + sum;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tmem_st16(tS + 16 * i, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * i]));
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * cc, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tO + 32 * cc, o);
+        }
+      }
+      m_ref = m_new;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar_p[k]);
+    }
+    if (ok && n > 0 && __all_sync(0xffffffffu, mbar_wait(&bar_o[k], 0, abort_flag, tmo, 122 + k))) {
+      tc_fence_after();
+      const float inv_l = 1.0f / l;
+      __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * N + q_row) * D;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32 * cc, o);
+        tmem_wait_ld();
+        if (q_row < N) {
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * cc);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
+      }
+      if (q_row < N) p.lse[static_cast<size_t>(bh) * N + q_row] = m_ref * p.scale + __logf(l);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace exattn

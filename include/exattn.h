@@ -1,0 +1,143 @@
+/*
+ * exattn — exact scaled-dot-product attention for NVIDIA B200 (sm_100a).
+ *
+ * What it computes.  For every batch b and head h:
+ *
+ *     S = scale * Q K^T,   P = softmax(S) row by row,   O = P V,
+ *
+ * the definition in "11.11 Flash Attention" (algomaster.io), section
+ * "Standard Attention: Step by Step" (Attention(Q,K,V) = softmax(Q K^T /
+ * sqrt(d_k)) V).  It is computed tile by tile with an online softmax (same
+ * page, sections "Flash Attention: The Key Insight" and "The Tiling
+ * Algorithm"), so the N x N matrices S and P never reach device memory.
+ * The forward also writes the per-row logsumexp
+ *
+ *     LSE_i = ln sum_j exp(S_ij),
+ *
+ * the per-row maximum m and running sum l of "Walk through the
+ * FlashAttention algorithm ..." (zenaique.com), answer to "How does the
+ * backward pass avoid storing the n x n attention matrix?", folded into one
+ * number.  The backward recomputes P from Q, K and LSE tile by tile ("11.11
+ * Flash Attention", section "The Recomputation Trade-off") and returns dQ, dK
+ * and dV, the chain rule of the definition above:
+ *
+ *     dV = P^T dO,  dP = dO V^T,  D_i = sum_k dO_ik O_ik,
+ *     dS = P o (dP - D 1^T),  dQ = scale dS K,  dK = scale dS^T Q.
+ *
+ * Conventions shared by every entry point
+ * ----------------------------------------
+ *  - Tensors q, k, v, o, dO, dq, dk, dv are bf16 (passed as raw 16-bit
+ *    patterns), contiguous, row-major [B, H, N, d]: the (batch, heads,
+ *    seq_len, head_dim) order of the pages' PyTorch examples.  lse is fp32
+ *    [B, H, N].  All of them are DEVICE pointers on the current CUDA device.
+ *  - d must be 64 or 128.  N >= 1 is arbitrary (no multiple-of-tile rule).
+ *    B, H or N equal to 0 is an empty problem: the call returns
+ *    ATTN_OK and touches nothing (pointers may then be NULL).
+ *  - causal != 0 applies the square top-left mask: query i sees key j iff
+ *    j <= i.  (The pages do not discuss masking; this is the usual reading.)
+ *  - scale is the softmax scale (1/sqrt(d) in the pages' formula); it must be
+ *    finite and > 0.
+ *  - Every pointer must be 16-byte aligned.  Outputs must not overlap inputs.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream).  They never synchronise and never allocate device
+ *    memory: the caller owns every buffer, including the backward workspace.
+ *  - Return value: an attn_status code.  Argument errors are detected on the
+ *    host before anything is launched.  A kernel that gives up waiting on an
+ *    internal barrier (a bounded wait of about one second; it should never
+ *    happen) records ATTN_ERR_TIMEOUT in a device status word that
+ *    attn_get_device_status() reports.
+ */
+#ifndef EXATTN_H_
+#define EXATTN_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* attn_stream_t;
+
+typedef enum attn_status {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID = 1,            /* bad argument: null/misaligned pointer, negative size,
+                                      d not in {64,128}, scale not finite or <= 0,
+                                      workspace too small, size overflow */
+  ATTN_ERR_UNSUPPORTED_DEVICE = 2, /* current device is not sm_100 (B200) */
+  ATTN_ERR_LAUNCH = 3,             /* a CUDA call failed (launch, attribute, tensor map) */
+  ATTN_ERR_TIMEOUT = 4             /* a device-side wait ran out (see above) */
+} attn_status;
+
+/*
+ * Forward pass.
+ *   q, k, v : in,  bf16 [B,H,N,d]
+ *   o       : out, bf16 [B,H,N,d]   O = softmax(scale Q K^T [+ mask]) V
+ *   lse     : out, fp32 [B,H,N]     natural-log logsumexp of each scaled score row
+ * Work: 4*d flops per unmasked (query, key) pair.
+ */
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+             float scale, int causal, attn_stream_t stream);
+
+/*
+ * Size in bytes of the device workspace attn_bwd() needs: an fp32 dQ
+ * accumulator [B,H,Np,d] plus fp32 D and pre-scaled LSE rows [B,H,Np], where
+ * Np is N rounded up to a multiple of 128.  Returns 0 for an empty or invalid
+ * problem.
+ */
+size_t attn_bwd_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * Backward pass: the three stages below, in order, on `stream`.
+ *   q, k, v, o, dO : in,  bf16 [B,H,N,d] (o from attn_fwd on the same inputs)
+ *   lse            : in,  fp32 [B,H,N]   (from attn_fwd)
+ *   dq, dk, dv     : out, bf16 [B,H,N,d]
+ *   workspace      : scratch, device, >= attn_bwd_workspace_bytes(B,H,N,d)
+ *                    bytes, 256-byte aligned; contents on entry are ignored.
+ * Work: 10*d flops per unmasked pair (five matmuls, one of them the
+ * recomputation of Q K^T).
+ */
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+             void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, void* workspace,
+             size_t workspace_bytes, attn_stream_t stream);
+
+/*
+ * The backward's stages, callable one by one (attn_bwd calls exactly these).
+ *
+ * Stage 1: D_i = sum_k dO_ik O_ik (fp32) and the LSE rows pre-multiplied by
+ * log2(e) into the workspace (padded rows get D = 0 and LSE = +inf, which
+ * makes their probabilities exactly 0), and zero the fp32 dQ accumulator.
+ */
+int attn_bwd_preprocess(const void* o, const void* dO, const float* lse, int B, int H, int N, int d,
+                        void* workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
+ * Stage 2: for each key tile, recompute S^T and P^T tile by tile and
+ * accumulate dV = P^T dO and dK = scale dS^T Q (written as bf16 to dk, dv),
+ * and add each tile's dS K into the fp32 dQ accumulator of the workspace.
+ * Needs stage 1's workspace contents.
+ */
+int attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, int B, int H,
+                  int N, int d, float scale, int causal, void* workspace, size_t workspace_bytes,
+                  attn_stream_t stream);
+
+/* Stage 3: dq = bf16(scale * dQ accumulator). */
+int attn_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, const void* workspace,
+                        size_t workspace_bytes, attn_stream_t stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device status word of
+ * the current device: ATTN_OK, or ATTN_ERR_TIMEOUT if any kernel of this
+ * library gave up waiting since the last call (ATTN_ERR_LAUNCH if the
+ * synchronisation itself failed).
+ */
+int attn_get_device_status(attn_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char* attn_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXATTN_H_ */

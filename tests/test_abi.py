@@ -1,0 +1,82 @@
+"""The C-ABI library: loads without a GPU, exports every declared symbol, and
+rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_attention_106_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "exattn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    assert declared_functions() == sorted(_lib.SIGNATURES)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    raw = ctypes.CDLL(_lib.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(raw, name), name
+
+
+def test_status_strings(lib):
+    assert _lib.status_string(0) == "ATTN_OK"
+    assert _lib.status_string(4) == "ATTN_ERR_TIMEOUT"
+    assert _lib.status_string(99) == "ATTN_ERR_UNKNOWN"
+
+
+P = 1 << 20  # a fake, 16-byte aligned "device" address; never dereferenced
+
+
+def fwd(lib, **kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, B=1, H=1, N=8, d=64, scale=0.125, causal=0, stream=None)
+    a.update(kw)
+    return lib.attn_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["N"], a["d"],
+                        a["scale"], a["causal"], a["stream"])
+
+
+@pytest.mark.parametrize("kw", [
+    dict(d=96), dict(d=256), dict(B=-1), dict(N=-5), dict(scale=0.0), dict(scale=-1.0),
+    dict(scale=float("inf")), dict(scale=float("nan")), dict(q=None), dict(lse=None),
+    dict(k=P + 8), dict(o=P + 2),
+])
+def test_fwd_rejects_bad_arguments_on_host(lib, kw):
+    assert fwd(lib, **kw) == _lib.ATTN_ERR_INVALID
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(H=0), dict(N=0), dict(N=0, q=None, o=None)])
+def test_empty_problem_is_a_no_op(lib, kw):
+    assert fwd(lib, **kw) == _lib.ATTN_OK
+
+
+def test_workspace_size(lib):
+    assert lib.attn_bwd_workspace_bytes(1, 1, 1, 64) == (128 * 64 + 2 * 128) * 4
+    assert lib.attn_bwd_workspace_bytes(2, 3, 129, 128) == 6 * (256 * 128 + 2 * 256) * 4
+    assert lib.attn_bwd_workspace_bytes(1, 1, 8, 80) == 0
+    assert lib.attn_bwd_workspace_bytes(0, 1, 8, 64) == 0
+
+
+def test_bwd_rejects_small_workspace_and_misalignment(lib):
+    need = lib.attn_bwd_workspace_bytes(1, 2, 300, 128)
+    args = [P] * 9 + [1, 2, 300, 128, 0.1, 1]
+    assert lib.attn_bwd(*args, P, need - 1, None) == _lib.ATTN_ERR_INVALID
+    assert lib.attn_bwd(*args, P + 16, need, None) == _lib.ATTN_ERR_INVALID  # workspace not 256-aligned
+    assert lib.attn_bwd_preprocess(P, P, P, 1, 2, 300, 128, P, need - 4, None) == _lib.ATTN_ERR_INVALID
+    assert lib.attn_bwd_dkdv(P, P, P, P, P, P, 1, 2, 300, 128, 0.1, 1, P, 0, None) == _lib.ATTN_ERR_INVALID
+    assert lib.attn_bwd_dq_convert(P, 1, 2, 300, 64, 0.0, P, need, None) == _lib.ATTN_ERR_INVALID
+    assert lib.attn_bwd(*([P] * 9), 0, 2, 300, 128, 0.1, 1, None, 0, None) == _lib.ATTN_OK
