@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "exattn.h"
 #include "ptx.cuh"
@@ -291,3 +292,53 @@ const char* attn_status_string(int status) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Backward with library-owned scratch: attn_bwd_noalloc().
+//
+// For callers that must not allocate device memory themselves: code that
+// runs with a fixed device-memory budget settled at start-up, plugins whose
+// host application owns the device allocator, and code paths where a
+// cudaMalloc/cudaFree (which may synchronise the whole device) is not
+// allowed.  The backward's scratch (fp32 dQ accumulator plus two fp32 row
+// vectors) lives in one file-scope __device__ array of
+// EXATTN_NOALLOC_SCRATCH_BYTES, which every GPU that loads this library holds
+// until the process exits.  In host code the array's name is only a host-side
+// stand-in, so its device address is fetched once per device with
+// cudaGetSymbolAddress (on the first call made with that device current) and
+// passed to the kernels.
+// ---------------------------------------------------------------------------
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[EXATTN_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices];  // device address of g_noalloc_scratch, per device; guarded by g_noalloc_mu
+
+int noalloc_scratch_address(int dev, void** out) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return ATTN_ERR_LAUNCH;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                                const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                                float scale, int causal, attn_stream_t stream) {
+  const int sz = check_sizes(B, H, N, d);
+  if (sz < 0 || !check_scale(scale)) return ATTN_ERR_INVALID;
+  if (sz == 1) return ATTN_OK;
+  if (workspace_bytes(B, H, N, d) > static_cast<size_t>(EXATTN_NOALLOC_SCRATCH_BYTES)) return ATTN_ERR_INVALID;
+  int dev = 0;
+  if (int st = check_device(&dev)) return st;
+  void* scratch = nullptr;
+  if (int st = noalloc_scratch_address(dev, &scratch)) return st;
+  return attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, scratch,
+                  static_cast<size_t>(EXATTN_NOALLOC_SCRATCH_BYTES), stream);
+}

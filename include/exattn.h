@@ -126,6 +126,37 @@ int attn_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, const
                         size_t workspace_bytes, attn_stream_t stream);
 
 /*
+ * Backward without any device allocation: attn_bwd() run on scratch memory
+ * that the library itself holds.  (The pages have no counterpart to this
+ * entry point; it exists for how callers manage memory, not for the method.)
+ *
+ * Meant for callers that cannot call cudaMalloc: code that must run within a
+ * device-memory budget fixed at start-up, plugins inside a host program that
+ * owns the device allocator, and code where an allocation, which can
+ * synchronise the whole device, is not allowed.  Such a caller still passes
+ * every input and output (same meaning, layout and rules as attn_bwd()); the
+ * workspace comes from one file-scope device array of
+ * EXATTN_NOALLOC_SCRATCH_BYTES (64 MiB) that every GPU which loads the
+ * library holds until the process exits.
+ *
+ *  - Problems whose attn_bwd_workspace_bytes(B,H,N,d) exceeds
+ *    EXATTN_NOALLOC_SCRATCH_BYTES are rejected with ATTN_ERR_INVALID before
+ *    anything runs: for d = 128 when B*H*ceil(N/128) > 1008, for d = 64
+ *    when B*H*ceil(N/128) > 1985.
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current); make that first call before any stream capture.
+ *  - Every call on a device shares the one array.  Each call re-initialises
+ *    the parts it reads, so leftover contents never leak into results, but
+ *    calls that overlap on the GPU (other streams, other host threads) race
+ *    on it: serialise them.
+ */
+#define EXATTN_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                     const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale,
+                     int causal, attn_stream_t stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word of
  * the current device: ATTN_OK, or ATTN_ERR_TIMEOUT if any kernel of this
  * library gave up waiting since the last call (ATTN_ERR_LAUNCH if the
