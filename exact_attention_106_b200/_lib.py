@@ -27,6 +27,8 @@ SIGNATURES = {
     "attn_bwd_dkdv": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _sz, _vp]),
     "attn_bwd_dq_convert": (_i, [_vp, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
     "attn_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp]),
+    "attn_set_wait_timeout_ns": (None, [ctypes.c_ulonglong]),
+    "attn_debug_inject_stall": (None, [_i]),
     "attn_get_device_status": (_i, [_vp]),
     "attn_status_string": (ctypes.c_char_p, [_i]),
 }

@@ -39,10 +39,12 @@ struct BwdParams {
   int Np;
   int BH;
   int ntiles;  // ceil(N / 128)
+  int head_group;  // heads whose CTAs are scheduled together (L2 reuse of Q/dO/dQ)
   int causal;
   float scale;
   float scale_log2;
   unsigned long long timeout_ns;
+  unsigned int debug_flags;
 };
 
 template <int D>
@@ -110,9 +112,10 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
   const int lane = threadIdx.x & 31;
   const int N = p.N;
   const int T = p.ntiles;
-  // Key tile 0 first: under the causal mask it sees the most query tiles.
-  const int j = static_cast<int>(blockIdx.x) / p.BH;
-  const int bh = static_cast<int>(blockIdx.x) % p.BH;
+  // Key tile 0 first (under the causal mask it sees the most query tiles), a
+  // few heads at a time.
+  int j, bh;
+  grouped_order(static_cast<int>(blockIdx.x), p.ntiles, p.BH, p.head_group, j, bh);
   const int i0 = p.causal ? j : 0;
   const int n = T - i0;  // >= 1
 
@@ -151,11 +154,14 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
       prefetch_tensormap(&p.tm_k);
       prefetch_tensormap(&p.tm_v);
       prefetch_tensormap(&p.tm_do);
-      mbar_arrive_expect_tx(bar_kv, 2 * TILE);
+      const bool kv_issued = !(p.debug_flags & kDebugSkipFirstKV);  // else: injected stall
+      if (kv_issued) {
+        mbar_arrive_expect_tx(bar_kv, 2 * TILE);
 #pragma unroll
-      for (int c = 0; c < C::kChunks; ++c) {
-        tma_load_3d(sK + c * 16384, &p.tm_k, bar_kv, c * 64, j * 128, bh);
-        tma_load_3d(sV + c * 16384, &p.tm_v, bar_kv, c * 64, j * 128, bh);
+        for (int c = 0; c < C::kChunks; ++c) {
+          tma_load_3d(sK + c * 16384, &p.tm_k, bar_kv, c * 64, j * 128, bh);
+          tma_load_3d(sV + c * 16384, &p.tm_v, bar_kv, c * 64, j * 128, bh);
+        }
       }
       int last_par0 = -1, last_par1 = -1;  // parity of the last load into each stage
       bool ok = true;
@@ -178,8 +184,9 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
         bulk_load(sVec + st * 256 + 128, p.dvec + vrow, 512, &bar_qfull[st]);
         if (st == 0) last_par0 = static_cast<int>(ph); else last_par1 = static_cast<int>(ph);
       }
-      if (!ok) {
-        drain_wait(bar_kv, 0, 202);
+      // Let every copy issued so far land before the CTA can exit.
+      {
+        if (kv_issued) drain_wait(bar_kv, 0, 202);
         if (last_par0 >= 0) drain_wait(&bar_qfull[0], static_cast<uint32_t>(last_par0), 203);
         if (last_par1 >= 0) drain_wait(&bar_qfull[1], static_cast<uint32_t>(last_par1), 203);
       }

@@ -21,6 +21,8 @@ using exattn::FwdParams;
 
 constexpr unsigned long long kDefaultTimeoutNs = 1000000000ull;  // 1 s per wait
 constexpr int kMaxDevices = 64;
+std::atomic<unsigned long long> g_timeout_ns{kDefaultTimeoutNs};  // see attn_set_wait_timeout_ns
+std::atomic<unsigned int> g_debug_flags{0};                        // see attn_debug_inject_stall
 
 // ------------------------------------------------------------------ checks
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -122,6 +124,15 @@ std::atomic<int> g_bwd128_attr[kMaxDevices];
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH; }
 
+// Heads per scheduling group: the CTAs in flight then touch about
+// kL2GroupBytes of per-head data, so that two groups fit in the 126 MB L2.
+constexpr double kL2GroupBytes = 48.0 * 1024 * 1024;
+int head_group(int BH, double per_head_bytes) {
+  const double g = kL2GroupBytes / per_head_bytes;
+  if (g >= BH) return BH;
+  return g < 1.0 ? 1 : static_cast<int>(g);
+}
+
 }  // namespace
 
 extern "C" {
@@ -148,10 +159,12 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.N = N;
   p.BH = BH;
   p.nblocks = (N + 255) / 256;
+  p.head_group = head_group(BH, 2.0 * N * d * 2);  // K and V of one head
   p.causal = causal ? 1 : 0;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.timeout_ns = kDefaultTimeoutNs;
+  p.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
+  p.debug_flags = g_debug_flags.load(std::memory_order_relaxed);
   const dim3 grid(static_cast<unsigned>(p.nblocks) * static_cast<unsigned>(BH));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 64) {
@@ -220,10 +233,12 @@ int attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, v
   p.Np = static_cast<int>(padded_rows(N));
   p.BH = BH;
   p.ntiles = (N + 127) / 128;
+  p.head_group = head_group(BH, 2.0 * N * d * 2 + 4.0 * N * d);  // Q, dO (bf16) and the dQ rows (fp32)
   p.causal = causal ? 1 : 0;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.timeout_ns = kDefaultTimeoutNs;
+  p.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
+  p.debug_flags = g_debug_flags.load(std::memory_order_relaxed);
   const dim3 grid(static_cast<unsigned>(p.ntiles) * static_cast<unsigned>(BH));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 64) {
@@ -267,6 +282,14 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
   st = attn_bwd_dkdv(q, k, v, dO, dk, dv, B, H, N, d, scale, causal, workspace, workspace_bytes_given, stream);
   if (st) return st;
   return attn_bwd_dq_convert(dq, B, H, N, d, scale, workspace, workspace_bytes_given, stream);
+}
+
+void attn_set_wait_timeout_ns(unsigned long long ns) {
+  g_timeout_ns.store(ns == 0 ? kDefaultTimeoutNs : ns, std::memory_order_relaxed);
+}
+
+void attn_debug_inject_stall(int on) {
+  g_debug_flags.store(on ? exattn::kDebugSkipFirstKV : 0u, std::memory_order_relaxed);
 }
 
 int attn_get_device_status(attn_stream_t stream) {

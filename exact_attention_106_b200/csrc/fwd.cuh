@@ -35,11 +35,18 @@ struct FwdParams {
   int N;
   int BH;
   int nblocks;  // ceil(N / 256)
+  int head_group;  // heads whose CTAs are scheduled together (L2 reuse of K/V)
   int causal;
   float scale;       // softmax scale
   float scale_log2;  // scale * log2(e)
   unsigned long long timeout_ns;
+  unsigned int debug_flags;
 };
+
+// Exponential pairs (out of every 8) evaluated by ex2_fma on the FMA pipe;
+// the special-function unit alone cannot keep pace with the tensor core at
+// d = 128 (one exp per score against 4*d flops of MMA).
+constexpr int kEmuPairs = 3;
 
 template <int D>
 struct FwdCfg {
@@ -81,9 +88,11 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_kernel(const __grid_constant_
   const int lane = threadIdx.x & 31;
   const int N = p.N;
   const int T = (N + 127) >> 7;
-  // Heaviest query blocks first (they see the most keys under the causal mask).
-  const int qb = p.nblocks - 1 - static_cast<int>(blockIdx.x) / p.BH;
-  const int bh = static_cast<int>(blockIdx.x) % p.BH;
+  // Heaviest query blocks first (they see the most keys under the causal
+  // mask), a few heads at a time.
+  int rank, bh;
+  grouped_order(static_cast<int>(blockIdx.x), p.nblocks, p.BH, p.head_group, rank, bh);
+  const int qb = p.nblocks - 1 - rank;
   int n_sub[2];
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
@@ -143,6 +152,7 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_kernel(const __grid_constant_
             ok = false;
             break;
           }
+          if (idx == 0 && (p.debug_flags & kDebugSkipFirstKV)) continue;  // injected stall
           mbar_arrive_expect_tx(&bar_full[slot], TILE);
           const CUtensorMap* m = x ? &p.tm_v : &p.tm_k;
 #pragma unroll
@@ -153,7 +163,10 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_kernel(const __grid_constant_
             if (s == slot) last_par[s] = static_cast<int>(ph);
         }
       }
-      if (!ok) {  // error path: let the copies already in flight land
+      // Let every copy issued so far land before the CTA can exit (on the
+      // normal path these phases have long completed; after an abort by any
+      // role some may still be in flight).
+      {
         drain_wait(bar_q, 0, 102);
 #pragma unroll
         for (int s = 0; s < SLOTS; ++s)
@@ -270,34 +283,49 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_kernel(const __grid_constant_
       tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
       tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
       tmem_wait_ld();
-      float s[128];
-#pragma unroll
-      for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(sr[i]);
       const int key0 = j * 128;
       const bool diag = p.causal && (j == 2 * qb + k);
       if (diag || key0 + 128 > N) {
         const int lim = min(diag ? row : 127, N - 1 - key0);  // last visible column
 #pragma unroll
         for (int i = 0; i < 128; ++i)
-          if (i > lim) s[i] = -INFINITY;
+          if (i > lim) sr[i] = __float_as_uint(-INFINITY);
       }
-      float mx = s[0];
+      // row maximum: four independent chains of 3-input max
+      float mxa[4];
 #pragma unroll
-      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+      for (int t = 0; t < 4; ++t) mxa[t] = __uint_as_float(sr[t]);
+#pragma unroll
+      for (int i = 4; i < 128; i += 2)
+        mxa[(i >> 1) & 3] = max3f(mxa[(i >> 1) & 3], __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]));
+      const float mx = fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3]));
       const float m_new = (mx > m_ref + thr) ? mx : m_ref;
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
       const float alpha = ex2((m_ref - m_use) * c);
-      const float neg = -m_use * c;
-      float sum = 0.f;
+      const uint64_t c2 = f2_pack(c, c);
+      const uint64_t neg2 = f2_pack(-m_use * c, -m_use * c);
+      uint64_t suma[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
       uint32_t pk[64];
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
-        const float p0 = ex2(fmaf(s[2 * i], c, neg));
-        const float p1 = ex2(fmaf(s[2 * i + 1], c, neg));
-        sum += p0 + p1;
+        const uint64_t x = f2_fma(f2_pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), c2, neg2);
+        uint64_t pp;
+        if ((i & 7) >= 8 - kEmuPairs) {  // kEmuPairs of every 8 pairs on the FMA pipe
+          pp = ex2_fma2(x);
+        } else {
+          float x0, x1;
+          f2_unpack(x, x0, x1);
+          pp = f2_pack(ex2(x0), ex2(x1));
+        }
+        suma[i & 1] = f2_add(suma[i & 1], pp);
+        float p0, p1;
+        f2_unpack(pp, p0, p1);
         pk[i] = pack_bf16x2(p0, p1);
       }
-      l = l * alpha + sum;
+      float s0, s1, s2, s3;
+      f2_unpack(suma[0], s0, s1);
+      f2_unpack(suma[1], s2, s3);
+      l = l * alpha + ((s0 + s1) + (s2 + s3));
 #pragma unroll
       for (int i = 0; i < 4; ++i) tmem_st16(tS + 16 * i, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * i]));
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {

@@ -22,6 +22,10 @@ enum : unsigned int {
   kDevStatusBadSmemAlign = 2u,
 };
 
+// Fault injection (see attn_debug_inject_stall): the producer skips its first
+// K/V load, so a consumer waits on a barrier that nothing will complete.
+enum : unsigned int { kDebugSkipFirstKV = 1u };
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -74,16 +78,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
                                           uint64_t timeout_ns, unsigned int site) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
+  // try_wait itself may suspend the thread for a while, so the clock and the
+  // abort flag are checked after every poll.
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
+  for (;;) {
     if (mbar_try_wait(a, parity)) return true;
-    if ((it & 63u) == 0u) {
-      if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > timeout_ns) {
-        record_status(kDevStatusTimeout, site);
-        *abort_flag = 1;
-        return false;
-      }
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > timeout_ns) {
+      record_status(kDevStatusTimeout, site);
+      *abort_flag = 1;
+      return false;
     }
   }
 }
@@ -234,6 +238,96 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// ------------------------------------------------- packed fp32 pairs (sm_100)
+// Two fp32 values in one 64-bit register pair; one instruction operates on
+// both, halving the issue cost of the softmax's scale, sum and polynomial.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add_rm(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x on the FMA pipe instead of the special-function unit:
+// 2^x = 2^n * p(f), n = floor(x), f = x - n in [0, 1), with p the degree-3
+// minimax (relative error) polynomial for 2^f with p(0) = 1, p(1) = 2, fitted
+// by csrc/gen_exp2_poly.py (max relative error 1.03e-4 in fp32).  floor(x)
+// comes from adding 1.5 * 2^23 with round-down; the exponent is added to p's
+// bits as an integer.  x is clamped to -127, where the result is exactly 0.
+__device__ __forceinline__ float ex2_fma(float x) {
+  x = fmaxf(x, -127.0f);
+  const float r = __fadd_rd(x, 12582912.0f);  // 1.5 * 2^23 + floor(x), exactly
+  const float f = x - (r - 12582912.0f);
+  const float p = fmaf(fmaf(fmaf(0.07826796919107437f, f, 0.226307675242424f), f, 0.6954243183135986f), f, 1.0f);
+  // low bits of r hold floor(x) (offset by 2^22, which shifts out)
+  return __int_as_float(__float_as_int(p) + (__float_as_int(r) << 23));
+}
+
+// ex2_fma on a packed pair (same arithmetic, half the instructions).
+__device__ __forceinline__ uint64_t ex2_fma2(uint64_t x) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  x = f2_pack(fmaxf(x0, -127.0f), fmaxf(x1, -127.0f));
+  const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
+  const uint64_t r = f2_add_rm(x, magic);
+  const uint64_t f = f2_sub(x, f2_sub(r, magic));
+  uint64_t q = f2_fma(f2_pack(0.07826796919107437f, 0.07826796919107437f), f,
+                      f2_pack(0.226307675242424f, 0.226307675242424f));
+  q = f2_fma(q, f, f2_pack(0.6954243183135986f, 0.6954243183135986f));
+  q = f2_fma(q, f, f2_pack(1.0f, 1.0f));
+  float q0, q1, r0, r1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(r, r0, r1);
+  return f2_pack(__int_as_float(__float_as_int(q0) + (__float_as_int(r0) << 23)),
+                 __int_as_float(__float_as_int(q1) + (__float_as_int(r1) << 23)));
+}
+
+// Maps a linear CTA index to (tile rank, head) so that the CTAs in flight
+// cover only a few heads at a time (their K/V, Q/dO and dQ rows then stay in
+// L2), and so that inside each group of `group` heads the heaviest tiles
+// (rank 0) start first.
+__device__ __forceinline__ void grouped_order(int bid, int ntile, int BH, int group, int& rank, int& bh) {
+  const int full = BH / group;
+  const int per_group = group * ntile;
+  int g = bid / per_group;
+  int gsz = group;
+  int rem = bid - g * per_group;
+  if (g >= full) {  // trailing group with fewer heads
+    g = full;
+    gsz = BH - full * group;
+    rem = bid - full * per_group;
+  }
+  rank = rem / gsz;
+  bh = g * group + rem % gsz;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

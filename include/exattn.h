@@ -164,6 +164,29 @@ int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
  */
 int attn_get_device_status(attn_stream_t stream);
 
+/*
+ * Failure detection.  Every wait of a kernel on one of its internal barriers
+ * is limited in time (1 s by default).  When a limit runs out the kernel
+ * records ATTN_ERR_TIMEOUT for attn_get_device_status(), all of its roles
+ * leave their loops, copies and matrix multiplies already in flight are
+ * allowed to finish, and the kernel returns: it never hangs the GPU, and the
+ * CUDA context stays usable.  This sets the limit used by launches made after
+ * the call, process-wide; 0 restores the default.  A limit of a few
+ * nanoseconds makes ordinary waits run out, which is how the failure path is
+ * tested.  (The pages have no counterpart; this is an operational control.)
+ */
+void attn_set_wait_timeout_ns(unsigned long long ns);
+
+/*
+ * Fault injection for testing the path above.  While `on` is nonzero, the
+ * forward and main backward kernels launched afterwards skip their first K/V
+ * tile load, so one of their roles waits on a barrier that nothing will ever
+ * complete; the bounded wait then runs out and the call reports
+ * ATTN_ERR_TIMEOUT (results are then undefined).  No fault, trap or hang is
+ * involved.  Off by default; process-wide.
+ */
+void attn_debug_inject_stall(int on);
+
 /* Static, human-readable name of a status code. */
 const char* attn_status_string(int status);
 

@@ -1,0 +1,46 @@
+"""Failure detection without a GPU fault.
+
+Every wait of the kernels on their internal barriers is limited in time.  Here
+the kernels are told to skip their first K/V load, so one role waits on a
+barrier that nothing completes, with the limit set to 20 ms: the kernels must
+record ATTN_ERR_TIMEOUT, leave their loops, let in-flight copies and MMAs
+finish and return, and the CUDA context must stay usable (a correct run right
+after, with injection off and the limit restored, matches the oracle).
+Nothing here faults, traps or hangs the GPU.
+"""
+import math
+
+import pytest
+import torch
+
+import exact_attention_106_b200 as ex
+from exact_attention_106_b200 import _lib
+from parity_util import check_all, oracle_ref, run_cuda
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_wait_limit_runs_out_and_context_survives(cuda_device, d):
+    lib = _lib.load()
+    g = torch.Generator().manual_seed(d)
+    q, k, v, do = (torch.randn((1, 2, 700, d), generator=g).bfloat16() for _ in range(4))
+    qd, kd, vd, dod = (x.to(cuda_device) for x in (q, k, v, do))
+    assert ex.device_status() == 0
+    lib.attn_set_wait_timeout_ns(20_000_000)
+    lib.attn_debug_inject_stall(1)
+    try:
+        o, lse = ex.forward(qd, kd, vd, causal=True)
+        st_fwd = ex.device_status()
+        ex.backward(qd, kd, vd, o, lse, dod, causal=True)
+        st_bwd = ex.device_status()
+    finally:
+        lib.attn_debug_inject_stall(0)
+        lib.attn_set_wait_timeout_ns(0)
+    assert st_fwd == _lib.ATTN_ERR_TIMEOUT
+    assert st_bwd == _lib.ATTN_ERR_TIMEOUT
+    assert ex.device_status() == 0  # the status word was cleared by the read
+    scale = 1 / math.sqrt(d)
+    got = run_cuda(q, k, v, do, True, scale)
+    ref = oracle_ref(q, k, v, do, True, scale)
+    check_all(got, ref, what=f"after timeout d={d}")
