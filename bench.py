@@ -356,7 +356,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="long_context_1x32x16384x128_causal")
-    ap.add_argument("--cpu-heads", type=int, default=2, help="full heads timed for cpu_baseline")
+    ap.add_argument("--cpu-heads", type=int, default=3, help="full heads timed for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=2048, help="oracle sample size per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
