@@ -34,8 +34,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 METRIC = "attention fwd/bwd TFLOP/s (bf16, d=128, N 1k-32k) and % of B200 BF16 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_bwd_dkdv_long_context_traffic.txt")
-KERNEL_SOURCES = [os.path.join(ROOT, "exact_attention_106_b200", "csrc", f)
-                  for f in ("bwd.cuh", "fwd.cuh", "ptx.cuh")]
+KERNEL_SOURCES = [os.path.join(ROOT, "exact_attention_106_b200", "csrc", f) for f in ("bwd.cuh", "ptx.cuh")]
 
 
 # --------------------------------------------------------------------- utils
