@@ -138,6 +138,12 @@ def reduce_max(value: float, device) -> float:
     return float(t.item())
 
 
+def job_throughput(world: int, flops_per_step: float, steps: int, max_ms: float) -> float:
+    """Whole-job TFLOP/s: every rank processes `steps` steps of its own batch;
+    the time is the slowest rank's."""
+    return world * flops_per_step * steps / (max_ms * 1e-3) / 1e12
+
+
 def rank_workload(base, rank: int):
     """Each rank gets its own batch: same shape, seeds shifted by the rank."""
     import dataclasses
@@ -282,7 +288,7 @@ def run_ours(args, rank, world, local_rank):
     dominant = "bwd_dkdv" if mean["bwd_dkdv"] >= mean["fwd"] else "fwd"
     dom_tf = dkdv_tf if dominant == "bwd_dkdv" else fwd_tf
     peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
-    value = world * flops_step * args.steps / (max_ms * 1e-3) / 1e12
+    value = job_throughput(world, flops_step, args.steps, max_ms)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         v_cpu, dt_cpu, nh = time_oracle_heads(w, args.cpu_heads)
@@ -308,7 +314,7 @@ def run_ours(args, rank, world, local_rank):
                      "frac": dom_tf / peak, "peak_kind": f"bf16 sustained ({peak_src})",
                      "traffic": recorded_traffic() if dominant == "bwd_dkdv" else None},
         "cpu_baseline": cpu,
-        "e2e": {"value": world * flops_step * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": job_throughput(world, flops_step, e2e_steps, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "clocks": clk.summary(),
         "gpu_launches": 4 * args.steps,
