@@ -18,7 +18,9 @@
 //     dV_j += P^T dO_i           (A operand read from TMEM)
 //     dS^T = P^T o (dP^T - D_i)  (registers -> shared memory as bf16)
 //     dK_j += dS^T Q_i ;  dQ_i-partial = dS K_j  (tcgen05)
-//   and adds the dQ partial into the fp32 accumulator with vector reductions.
+//   and adds the dQ partial into the fp32 accumulator: four drain warps read
+//   it from tensor memory (handing the columns back at once), stage it in
+//   shared memory and let the TMA engine add it into global memory.
 // Stage 3 (attn_bwd_dq_convert_kernel): dQ = bf16(scale * accumulator).
 #pragma once
 #include "ptx.cuh"
@@ -30,6 +32,7 @@ struct BwdParams {
   CUtensorMap tm_k;
   CUtensorMap tm_v;
   CUtensorMap tm_do;
+  CUtensorMap tm_dq;  // fp32 2-D {d, B*H*Np}, box {32, 32}, 128-byte swizzle (dQ accumulator)
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   float* dq_acc;       // [BH, Np, d]
@@ -70,9 +73,16 @@ struct BwdCfg {
   static constexpr uint32_t kColDQ = (D == 128) ? kColDP : 384;  // d=128: dQ reuses dP's columns
 };
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
+// X[128 x 128] = A[128 x D] B[128 x D]^T with both operands K-major D-wide
+// tiles at offsets a0, b0 from the shared-memory base (S^T and dP^T).
+template <int D>
+__device__ __forceinline__ void bwd_issue_t(uint32_t d_tmem, SmemDesc dKm, uint32_t a0, uint32_t b0) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+    mma_ss(d_tmem, desc_at(dKm, a0 + off), desc_at(dKm, b0 + off), idesc, kk > 0 ? 1u : 0u);
+  }
 }
 
 template <int D>
@@ -100,7 +110,7 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
   uint64_t* bar_dp = bars + 6;      // dP^T ready
   uint64_t* bar_p = bars + 7;       // P^T written (256 arrivals)
   uint64_t* bar_ds = bars + 8;      // dS written to smem (256 arrivals)
-  uint64_t* bar_dsfree = bars + 9;  // dS smem consumed
+  uint64_t* bar_dsfree = bars + 9;  // dS smem free again (MMAs done, dQ staging read out; 4 arrivals)
   uint64_t* bar_dqfull = bars + 10; // dQ partial ready in TMEM
   uint64_t* bar_dqfree = bars + 11; // dQ partial read out (128 arrivals)
   uint64_t* bar_final = bars + 12;  // all MMAs done
@@ -129,7 +139,7 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
     mbar_init(bar_dp, 1);
     mbar_init(bar_p, 256);
     mbar_init(bar_ds, 256);
-    mbar_init(bar_dsfree, 1);
+    mbar_init(bar_dsfree, 4);
     mbar_init(bar_dqfull, 1);
     mbar_init(bar_dqfree, 128);
     mbar_init(bar_final, 1);
@@ -195,26 +205,20 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_t = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T: both operands K-major
       constexpr uint32_t idesc_kv = idesc_bf16_f32(128, D, 0, 1);   // dV, dK: B = dO / Q MN-major
       constexpr uint32_t idesc_q = idesc_bf16_f32(128, D, 1, 1);    // dQ: A = dS MN-major, B = K MN-major
-      const uint32_t sK0 = smem_u32(sK), sV0 = smem_u32(sV), sQ0 = smem_u32(sQ), sDO0 = smem_u32(sDO);
-      const uint32_t sDS0 = smem_u32(sDS);
-      // X[128 x 128] = A[128 x D] B[128 x D]^T, both K-major D-wide tiles
-      auto issue_t = [&](uint32_t dcol, uint32_t a0, uint32_t b0) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(tmem + dcol, smem_desc_sw128(a0 + off, 16, 1024), smem_desc_sw128(b0 + off, 16, 1024), idesc_t,
-                 kk > 0 ? 1u : 0u);
-        }
-      };
+      // K-major and MN-major views of this CTA's shared memory, built once;
+      // every operand below is an offset from the dynamic shared-memory base.
+      const SmemDesc dKm = make_desc_sw128(smem_u32(smem), 16, 1024);
+      const SmemDesc dMN = make_desc_sw128(smem_u32(smem), 16384, 1024);
+      constexpr uint32_t oK = C::kOffK, oV = C::kOffV, oQ = C::kOffQ, oDO = C::kOffDO, oDS = C::kOffDS;
+
       bool ok = mbar_wait(bar_kv, 0, abort_flag, tmo, 210) && mbar_wait(&bar_qfull[0], 0, abort_flag, tmo, 211);
       if (ok) {
         tc_fence_after();
-        issue_t(C::kColS, sK0, sQ0);
+        bwd_issue_t<D>(tmem + C::kColS, dKm, oK, oQ);
         tc_commit(bar_s);
-        issue_t(C::kColDP, sV0, sDO0);
+        bwd_issue_t<D>(tmem + C::kColDP, dKm, oV, oDO);
         tc_commit(bar_dp);
       }
       for (int it = 0; it < n && ok; ++it) {
@@ -226,14 +230,13 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ts(tmem + C::kColDV, tmem + C::kColS + (kk >> 2) * 64 + (kk & 3) * 8,
-                 smem_desc_sw128(sDO0 + st * TILE + kk * 2048, 16384, 1024), idesc_kv,
-                 (it > 0 || kk > 0) ? 1u : 0u);
+                 desc_at(dMN, oDO + st * TILE + kk * 2048), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
         // next S^T as early as possible: the softmax of tile it+1 overlaps dK, dQ of tile it
         if (it + 1 < n) {
           const int st1 = (it + 1) & 1;
           if (!mbar_wait(&bar_qfull[st1], ((it + 1) >> 1) & 1, abort_flag, tmo, 213)) break;
           tc_fence_after();
-          issue_t(C::kColS, sK0, sQ0 + st1 * TILE);
+          bwd_issue_t<D>(tmem + C::kColS, dKm, oK, oQ + st1 * TILE);
           tc_commit(bar_s);
         }
         if (!mbar_wait(bar_ds, it & 1, abort_flag, tmo, 214)) break;
@@ -242,8 +245,7 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t offa = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(tmem + C::kColDK, smem_desc_sw128(sDS0 + offa, 16, 1024),
-                 smem_desc_sw128(sQ0 + st * TILE + kk * 2048, 16384, 1024), idesc_kv,
+          mma_ss(tmem + C::kColDK, desc_at(dKm, oDS + offa), desc_at(dMN, oQ + st * TILE + kk * 2048), idesc_kv,
                  (it > 0 || kk > 0) ? 1u : 0u);
         }
         if (D != 128 && it > 0) {  // separate dQ columns: only the previous dQ must be drained
@@ -253,17 +255,16 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
         // dQ_i partial = dS K_j   (A = dS MN-major in smem, B = K_j MN-major)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + C::kColDQ, smem_desc_sw128(sDS0 + kk * 2048, 16384, 1024),
-                 smem_desc_sw128(sK0 + kk * 2048, 16384, 1024), idesc_q, kk > 0 ? 1u : 0u);
-        tc_commit(bar_dqfull);
+          mma_ss(tmem + C::kColDQ, desc_at(dMN, oDS + kk * 2048), desc_at(dMN, oK + kk * 2048), idesc_q,
+                 kk > 0 ? 1u : 0u);
+        tc_commit(bar_dqfull);  // also tells the drain that dK and dQ no longer read dS
         tc_commit(&bar_qempty[st]);
-        tc_commit(bar_dsfree);
         if (it + 1 < n) {
           if (D == 128) {  // dP^T(it+1) overwrites the dQ partial: wait until it is read out
             if (!mbar_wait(bar_dqfree, it & 1, abort_flag, tmo, 216)) break;
             tc_fence_after();
           }
-          issue_t(C::kColDP, sV0, sDO0 + ((it + 1) & 1) * TILE);
+          bwd_issue_t<D>(tmem + C::kColDP, dKm, oV, oDO + ((it + 1) & 1) * TILE);
           tc_commit(bar_dp);
         }
       }
@@ -377,28 +378,67 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
     }
   } else if (warp < 12) {
     // ------------------------------------------------------------ dQ drain
+    // Warp w owns query rows [32 w, 32 w + 32) of the partial.  Columns go in
+    // 64-wide passes through an 8 KB slice of the dS buffer (free once the dK
+    // and dQ MMAs that read dS are done, i.e. once the partial is ready), laid
+    // out as two 32-column TMA boxes with 128-byte swizzle; one lane then
+    // issues the TMA reduce-adds into the fp32 accumulator.
     const int wq = warp & 3;
-    const int r = wq * 32 + lane;  // query row in the tile
     const uint32_t tQ = tmem + (static_cast<uint32_t>(wq * 32) << 16) + C::kColDQ;
+    uint8_t* stage = sDS + wq * 8192;
+    uint8_t* my_row = stage + lane * 128;
+    const uint32_t swz = static_cast<uint32_t>(lane & 7);
+    auto stage_pass = [&](const uint32_t (&a)[32], const uint32_t (&b)[32]) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        *reinterpret_cast<uint4*>(my_row + ((u ^ swz) << 4)) = make_uint4(a[4 * u], a[4 * u + 1], a[4 * u + 2], a[4 * u + 3]);
+        *reinterpret_cast<uint4*>(my_row + 4096 + ((u ^ swz) << 4)) =
+            make_uint4(b[4 * u], b[4 * u + 1], b[4 * u + 2], b[4 * u + 3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+    };
     for (int it = 0; it < n; ++it) {
       if (!__all_sync(0xffffffffu, mbar_wait(bar_dqfull, it & 1, abort_flag, tmo, 230))) break;
       tc_fence_after();
-      float* dst = p.dq_acc + (static_cast<size_t>(bh) * p.Np + static_cast<size_t>(i0 + it) * 128 + r) * D;
-#pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t a[32];
-        tmem_ld32(tQ + 32 * cc, a);
-        tmem_wait_ld();
-        if (cc == D / 32 - 1) {  // every read of this partial is complete: hand the columns back
-          tc_fence_before();
-          mbar_arrive(bar_dqfree);
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          red_add_v4(dst + 32 * cc + 4 * e, __uint_as_float(a[4 * e]), __uint_as_float(a[4 * e + 1]),
-                     __uint_as_float(a[4 * e + 2]), __uint_as_float(a[4 * e + 3]));
+      const int grow = bh * p.Np + (i0 + it) * 128 + wq * 32;  // first accumulator row of this warp
+      uint32_t a[32], b[32];
+      tmem_ld32(tQ, a);
+      tmem_ld32(tQ + 32, b);
+      tmem_wait_ld();
+      if (D == 64) {  // every read of this partial is complete: hand the columns back
+        tc_fence_before();
+        mbar_arrive(bar_dqfree);
       }
+      stage_pass(a, b);
+      if (lane == 0) {
+        tma_reduce_add_2d(stage, &p.tm_dq, 0, grow);
+        tma_reduce_add_2d(stage + 4096, &p.tm_dq, 32, grow);
+        bulk_commit_group();
+      }
+      if (D == 128) {
+        tmem_ld32(tQ + 64, a);
+        tmem_ld32(tQ + 96, b);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar_dqfree);
+        if (lane == 0) bulk_wait_group_read0();  // the first pass has left shared memory
+        __syncwarp();
+        stage_pass(a, b);
+        if (lane == 0) {
+          tma_reduce_add_2d(stage, &p.tm_dq, 64, grow);
+          tma_reduce_add_2d(stage + 4096, &p.tm_dq, 96, grow);
+          bulk_commit_group();
+        }
+      }
+      if (lane == 0) {
+        bulk_wait_group_read0();
+        mbar_arrive(bar_dsfree);  // the compute warps may write the next dS
+      }
+      __syncwarp();
     }
+    if (lane == 0) bulk_wait_group0();  // the additions have reached global memory
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();

@@ -107,6 +107,20 @@ bool make_map_bf16(CUtensorMap* m, const void* base, int BH, int N, int d) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D view {d, rows} of the fp32 dQ accumulator [rows, d]; box {32, 32} with
+// 128-byte swizzle, the target of the backward's TMA reduce-adds.
+bool make_map_f32_dq(CUtensorMap* m, void* base, size_t rows, int d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 4};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Per-device, per-kernel one-time opt-in to large dynamic shared memory.
 template <typename K>
 bool ensure_smem_attr(K kernel, int dev, std::atomic<int>* flags, int bytes) {
@@ -222,7 +236,8 @@ int attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, v
   std::memset(&p, 0, sizeof(p));
   const int BH = B * H;
   if (!make_map_bf16(&p.tm_q, q, BH, N, d) || !make_map_bf16(&p.tm_k, k, BH, N, d) ||
-      !make_map_bf16(&p.tm_v, v, BH, N, d) || !make_map_bf16(&p.tm_do, dO, BH, N, d))
+      !make_map_bf16(&p.tm_v, v, BH, N, d) || !make_map_bf16(&p.tm_do, dO, BH, N, d) ||
+      !make_map_f32_dq(&p.tm_dq, ws.dq_acc, static_cast<size_t>(BH) * padded_rows(N), d))
     return ATTN_ERR_LAUNCH;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);

@@ -185,25 +185,26 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_kernel(const __grid_constant_
       auto kph = [&](int j) { return static_cast<uint32_t>(((2 * j) / SLOTS) & 1); };
       auto vslot = [&](int j) { return (2 * j + 1) % SLOTS; };
       auto vph = [&](int j) { return static_cast<uint32_t>(((2 * j + 1) / SLOTS) & 1); };
+      // K-major view (Q, K) and MN-major view (V) of the tiles, built once
+      const SmemDesc dK = make_desc_sw128(sq0, 16, 1024);
+      const SmemDesc dMN = make_desc_sw128(skv0, 16384, 1024);
       auto issue_s = [&](int k, int slot) {
-        const uint32_t a0 = sq0 + k * TILE, b0 = skv0 + slot * TILE;
+        const uint32_t a0 = k * TILE;                   // Q_k, relative to sQ
+        const uint32_t b0 = (skv0 - sq0) + slot * TILE;  // K_j, relative to sQ
         const uint32_t dt = tmem + k * 256;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(dt, smem_desc_sw128(a0 + off, 16, 1024), smem_desc_sw128(b0 + off, 16, 1024), idesc_s,
-                 kk > 0 ? 1u : 0u);
+          mma_ss(dt, desc_at(dK, a0 + off), desc_at(dK, b0 + off), idesc_s, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int k, int slot, bool acc) {
-        const uint32_t b0 = skv0 + slot * TILE;
+        const uint32_t b0 = slot * TILE;  // V_j, relative to the ring
         const uint32_t dt = tmem + k * 256 + 128;
         const uint32_t at = tmem + k * 256;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          mma_ts(dt, at + kk * 8, smem_desc_sw128(b0 + kk * 2048, 16384, 1024), idesc_o,
-                 (acc || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(dt, at + kk * 8, desc_at(dMN, b0 + kk * 2048), idesc_o, (acc || kk > 0) ? 1u : 0u);
       };
       const int n0 = n_sub[0], n1 = n_sub[1];
       bool ok = mbar_wait(bar_q, 0, abort_flag, tmo, 110);
