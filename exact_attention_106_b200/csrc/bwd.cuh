@@ -63,7 +63,11 @@ struct BwdCfg {
   static constexpr uint32_t kOffDO = 4 * kTile;  // 2 stages
   static constexpr uint32_t kOffDS = 6 * kTile;  // 128 x 128 bf16
   static constexpr uint32_t kOffVec = kOffDS + 32768;  // 2 stages x (LSE2[128], D[128]) fp32
-  static constexpr uint32_t kOffBar = kOffVec + 2048;
+  // dQ staging: at d = 128 the dO buffer of the step being drained (dead once
+  // dV and dP have read it); at d = 64 a buffer of its own (32 KB).
+  static constexpr uint32_t kOffStage = kOffVec + 2048;
+  static constexpr uint32_t kStageBytes = (D == 128) ? 0u : 32768u;
+  static constexpr uint32_t kOffBar = kOffStage + kStageBytes;
   static constexpr uint32_t kSmem = kOffBar + 256;
   // tensor-memory columns
   static constexpr uint32_t kColDK = 0;
@@ -104,18 +108,20 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
   float* sVec = reinterpret_cast<float*>(smem + C::kOffVec);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* bar_kv = bars + 0;
-  uint64_t* bar_qfull = bars + 1;   // [2]
-  uint64_t* bar_qempty = bars + 3;  // [2]
-  uint64_t* bar_s = bars + 5;       // S^T ready
-  uint64_t* bar_dp = bars + 6;      // dP^T ready
-  uint64_t* bar_p = bars + 7;       // P^T written (256 arrivals)
-  uint64_t* bar_ds = bars + 8;      // dS written to smem (256 arrivals)
-  uint64_t* bar_dsfree = bars + 9;  // dS smem free again (MMAs done, dQ staging read out; 4 arrivals)
-  uint64_t* bar_dqfull = bars + 10; // dQ partial ready in TMEM
-  uint64_t* bar_dqfree = bars + 11; // dQ partial read out (128 arrivals)
-  uint64_t* bar_final = bars + 12;  // all MMAs done
-  uint64_t* bar_drain = bars + 13;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  uint64_t* bar_qfull = bars + 1;    // [2] Q_i, LSE_i, D_i landed
+  uint64_t* bar_qempty = bars + 3;   // [2] Q_i, LSE_i, D_i consumed (MMA commit after dK)
+  uint64_t* bar_dofull = bars + 5;   // [2] dO_i landed
+  uint64_t* bar_doempty = bars + 7;  // [2] dO_i buffer free (the drain warps, after their staging; 4 arrivals)
+  uint64_t* bar_s = bars + 9;        // S^T ready
+  uint64_t* bar_dp = bars + 10;      // dP^T ready
+  uint64_t* bar_p = bars + 11;       // P^T written (256 arrivals)
+  uint64_t* bar_ds = bars + 12;      // dS written to smem (256 arrivals)
+  uint64_t* bar_dsfree = bars + 13;  // dS consumed by the dQ and dK MMAs
+  uint64_t* bar_dqfull = bars + 14;  // dQ partial ready in TMEM
+  uint64_t* bar_dqfree = bars + 15;  // dQ partial read out of TMEM (128 arrivals)
+  uint64_t* bar_final = bars + 16;   // all MMAs done
+  uint64_t* bar_drain = bars + 17;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -134,12 +140,14 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar_qfull[s], 1);
       mbar_init(&bar_qempty[s], 1);
+      mbar_init(&bar_dofull[s], 1);
+      mbar_init(&bar_doempty[s], 4);
     }
     mbar_init(bar_s, 1);
     mbar_init(bar_dp, 1);
     mbar_init(bar_p, 256);
     mbar_init(bar_ds, 256);
-    mbar_init(bar_dsfree, 4);
+    mbar_init(bar_dsfree, 1);
     mbar_init(bar_dqfull, 1);
     mbar_init(bar_dqfree, 128);
     mbar_init(bar_final, 1);
@@ -173,47 +181,47 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
           tma_load_3d(sV + c * 16384, &p.tm_v, bar_kv, c * 64, j * 128, bh);
         }
       }
-      int last_par0 = -1, last_par1 = -1;  // parity of the last load into each stage
-      bool ok = true;
+      int lq[2] = {-1, -1}, ld[2] = {-1, -1};  // parity of the last loads into each stage
       for (int it = 0; it < n; ++it) {
         const int st = it & 1;
         const uint32_t ph = (it >> 1) & 1;
-        if (!mbar_wait(&bar_qempty[st], ph ^ 1u, abort_flag, tmo, 201)) {
-          ok = false;
-          break;
-        }
         const int i = i0 + it;
-        mbar_arrive_expect_tx(&bar_qfull[st], 2 * TILE + 1024);
+        if (!mbar_wait(&bar_qempty[st], ph ^ 1u, abort_flag, tmo, 201)) break;
+        mbar_arrive_expect_tx(&bar_qfull[st], TILE + 1024);
 #pragma unroll
-        for (int c = 0; c < C::kChunks; ++c) {
+        for (int c = 0; c < C::kChunks; ++c)
           tma_load_3d(sQ + st * TILE + c * 16384, &p.tm_q, &bar_qfull[st], c * 64, i * 128, bh);
-          tma_load_3d(sDO + st * TILE + c * 16384, &p.tm_do, &bar_qfull[st], c * 64, i * 128, bh);
-        }
         const size_t vrow = static_cast<size_t>(bh) * p.Np + static_cast<size_t>(i) * 128;
         bulk_load(sVec + st * 256, p.lse2 + vrow, 512, &bar_qfull[st]);
         bulk_load(sVec + st * 256 + 128, p.dvec + vrow, 512, &bar_qfull[st]);
-        if (st == 0) last_par0 = static_cast<int>(ph); else last_par1 = static_cast<int>(ph);
+        if (st == 0) lq[0] = static_cast<int>(ph); else lq[1] = static_cast<int>(ph);
+        if (!mbar_wait(&bar_doempty[st], ph ^ 1u, abort_flag, tmo, 202)) break;
+        mbar_arrive_expect_tx(&bar_dofull[st], TILE);
+#pragma unroll
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_3d(sDO + st * TILE + c * 16384, &p.tm_do, &bar_dofull[st], c * 64, i * 128, bh);
+        if (st == 0) ld[0] = static_cast<int>(ph); else ld[1] = static_cast<int>(ph);
       }
       // Let every copy issued so far land before the CTA can exit.
-      {
-        if (kv_issued) drain_wait(bar_kv, 0, 202);
-        if (last_par0 >= 0) drain_wait(&bar_qfull[0], static_cast<uint32_t>(last_par0), 203);
-        if (last_par1 >= 0) drain_wait(&bar_qfull[1], static_cast<uint32_t>(last_par1), 203);
+      if (kv_issued) drain_wait(bar_kv, 0, 203);
+      for (int s = 0; s < 2; ++s) {
+        if (lq[s] >= 0) drain_wait(&bar_qfull[s], static_cast<uint32_t>(lq[s]), 204);
+        if (ld[s] >= 0) drain_wait(&bar_dofull[s], static_cast<uint32_t>(ld[s]), 205);
       }
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_kv = idesc_bf16_f32(128, D, 0, 1);   // dV, dK: B = dO / Q MN-major
-      constexpr uint32_t idesc_q = idesc_bf16_f32(128, D, 1, 1);    // dQ: A = dS MN-major, B = K MN-major
+      constexpr uint32_t idesc_kv = idesc_bf16_f32(128, D, 0, 1);  // dV, dK: B = dO / Q MN-major
+      constexpr uint32_t idesc_q = idesc_bf16_f32(128, D, 1, 1);   // dQ: A = dS MN-major, B = K MN-major
       // K-major and MN-major views of this CTA's shared memory, built once;
       // every operand below is an offset from the dynamic shared-memory base.
       const SmemDesc dKm = make_desc_sw128(smem_u32(smem), 16, 1024);
       const SmemDesc dMN = make_desc_sw128(smem_u32(smem), 16384, 1024);
       constexpr uint32_t oK = C::kOffK, oV = C::kOffV, oQ = C::kOffQ, oDO = C::kOffDO, oDS = C::kOffDS;
-
-      bool ok = mbar_wait(bar_kv, 0, abort_flag, tmo, 210) && mbar_wait(&bar_qfull[0], 0, abort_flag, tmo, 211);
+      bool ok = mbar_wait(bar_kv, 0, abort_flag, tmo, 210) && mbar_wait(&bar_qfull[0], 0, abort_flag, tmo, 211) &&
+                mbar_wait(&bar_dofull[0], 0, abort_flag, tmo, 212);
       if (ok) {
         tc_fence_after();
         bwd_issue_t<D>(tmem + C::kColS, dKm, oK, oQ);
@@ -223,24 +231,36 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
       }
       for (int it = 0; it < n && ok; ++it) {
         const int st = it & 1;
+        const int st1 = (it + 1) & 1;
+        const uint32_t ph1 = ((it + 1) >> 1) & 1;
         // dV += P^T dO_i   (A = P^T from TMEM, K = 128 queries; queries 0..63
         // sit in columns [0,32) of the score block, 64..127 in [64,96))
-        if (!mbar_wait(bar_p, it & 1, abort_flag, tmo, 212)) break;
+        if (!mbar_wait(bar_p, it & 1, abort_flag, tmo, 213)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ts(tmem + C::kColDV, tmem + C::kColS + (kk >> 2) * 64 + (kk & 3) * 8,
                  desc_at(dMN, oDO + st * TILE + kk * 2048), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
-        // next S^T as early as possible: the softmax of tile it+1 overlaps dK, dQ of tile it
+        // next S^T as early as possible: the softmax of tile it+1 overlaps dQ, dK of tile it
         if (it + 1 < n) {
-          const int st1 = (it + 1) & 1;
-          if (!mbar_wait(&bar_qfull[st1], ((it + 1) >> 1) & 1, abort_flag, tmo, 213)) break;
+          if (!mbar_wait(&bar_qfull[st1], ph1, abort_flag, tmo, 214)) break;
           tc_fence_after();
           bwd_issue_t<D>(tmem + C::kColS, dKm, oK, oQ + st1 * TILE);
           tc_commit(bar_s);
         }
-        if (!mbar_wait(bar_ds, it & 1, abort_flag, tmo, 214)) break;
+        if (!mbar_wait(bar_ds, it & 1, abort_flag, tmo, 215)) break;
         tc_fence_after();
+        if (D != 128 && it > 0) {  // separate dQ columns: only the previous dQ must be drained
+          if (!mbar_wait(bar_dqfree, (it - 1) & 1, abort_flag, tmo, 216)) break;
+          tc_fence_after();
+        }
+        // dQ_i partial = dS K_j   (A = dS MN-major in smem, B = K_j MN-major),
+        // first, so that its drain overlaps dK
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + C::kColDQ, desc_at(dMN, oDS + kk * 2048), desc_at(dMN, oK + kk * 2048), idesc_q,
+                 kk > 0 ? 1u : 0u);
+        tc_commit(bar_dqfull);  // also: dV_i and dP_i, the readers of dO_i, are done
         // dK += dS^T Q_i   (A = dS^T K-major in smem, B = Q_i MN-major)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -248,29 +268,21 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
           mma_ss(tmem + C::kColDK, desc_at(dKm, oDS + offa), desc_at(dMN, oQ + st * TILE + kk * 2048), idesc_kv,
                  (it > 0 || kk > 0) ? 1u : 0u);
         }
-        if (D != 128 && it > 0) {  // separate dQ columns: only the previous dQ must be drained
-          if (!mbar_wait(bar_dqfree, (it - 1) & 1, abort_flag, tmo, 215)) break;
-          tc_fence_after();
-        }
-        // dQ_i partial = dS K_j   (A = dS MN-major in smem, B = K_j MN-major)
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + C::kColDQ, desc_at(dMN, oDS + kk * 2048), desc_at(dMN, oK + kk * 2048), idesc_q,
-                 kk > 0 ? 1u : 0u);
-        tc_commit(bar_dqfull);  // also tells the drain that dK and dQ no longer read dS
+        tc_commit(bar_dsfree);
         tc_commit(&bar_qempty[st]);
         if (it + 1 < n) {
           if (D == 128) {  // dP^T(it+1) overwrites the dQ partial: wait until it is read out
-            if (!mbar_wait(bar_dqfree, it & 1, abort_flag, tmo, 216)) break;
-            tc_fence_after();
+            if (!mbar_wait(bar_dqfree, it & 1, abort_flag, tmo, 217)) break;
           }
-          bwd_issue_t<D>(tmem + C::kColDP, dKm, oV, oDO + ((it + 1) & 1) * TILE);
+          if (!mbar_wait(&bar_dofull[st1], ph1, abort_flag, tmo, 218)) break;
+          tc_fence_after();
+          bwd_issue_t<D>(tmem + C::kColDP, dKm, oV, oDO + st1 * TILE);
           tc_commit(bar_dp);
         }
       }
       tc_commit(bar_final);
       tc_commit(bar_drain);
-      drain_wait(bar_drain, 0, 217);
+      drain_wait(bar_drain, 0, 219);
     }
     __syncwarp();
   } else if (warp < 8) {
@@ -301,19 +313,47 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
       tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
       tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_wait_ld();
-      const float* lse2 = sVec + st * 256 + 64 * h;
-      const float* dv = sVec + st * 256 + 128 + 64 * h;
+      const float4* lse4 = reinterpret_cast<const float4*>(sVec + st * 256 + 64 * h);
+      const float4* dv4 = reinterpret_cast<const float4*>(sVec + st * 256 + 128 + 64 * h);
       const bool diag = p.causal && (it == 0);
-      float pf[64];
+      // P^T = exp2(S^T c - LSE log2 e), in packed pairs; kEmuPairs of every 8
+      // pairs on the FMA pipe (ex2_fma2), the rest on the special-function unit
+      const uint64_t c2 = f2_pack(c, c);
+      uint64_t pf[32];
 #pragma unroll
-      for (int e = 0; e < 64; ++e) {
-        float pv = ex2(fmaf(__uint_as_float(sr[e]), c, -lse2[e]));
-        if (!key_ok || (diag && r > 64 * h + e)) pv = 0.f;
-        pf[e] = pv;
+      for (int q4 = 0; q4 < 16; ++q4) {
+        const float4 l4 = lse4[q4];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int e = 4 * q4 + 2 * hh;
+          const uint64_t nl = hh ? f2_pack(-l4.z, -l4.w) : f2_pack(-l4.x, -l4.y);
+          const uint64_t x = f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), c2, nl);
+          if (((e >> 1) & 7) >= 8 - kEmuPairs) {
+            pf[e >> 1] = ex2_fma2(x);
+          } else {
+            float x0, x1;
+            f2_unpack(x, x0, x1);
+            pf[e >> 1] = f2_pack(ex2(x0), ex2(x1));
+          }
+        }
+      }
+      if (!key_ok || diag) {  // the key is padding, or the tile is on the diagonal
+#pragma unroll
+        for (int e2 = 0; e2 < 32; ++e2) {
+          float p0, p1;
+          f2_unpack(pf[e2], p0, p1);
+          if (!key_ok || (diag && r > 64 * h + 2 * e2)) p0 = 0.f;
+          if (!key_ok || (diag && r > 64 * h + 2 * e2 + 1)) p1 = 0.f;
+          pf[e2] = f2_pack(p0, p1);
+        }
       }
       uint32_t pk[32];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(pf[2 * e], pf[2 * e + 1]);
+      for (int e2 = 0; e2 < 32; ++e2) {
+        float p0, p1;
+        f2_unpack(pf[e2], p0, p1);
+        pk[e2] = pack_bf16x2(p0, p1);
+      }
       tmem_st16(tP, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
       tmem_st16(tP + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
       tmem_wait_st();
@@ -336,11 +376,18 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
         tmem_wait_ld();
         uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int e0 = 32 * ch + 2 * e;
-          const float d0 = pf[e0] * (__uint_as_float(dpr[2 * e]) - dv[e0]);
-          const float d1 = pf[e0 + 1] * (__uint_as_float(dpr[2 * e + 1]) - dv[e0 + 1]);
-          w[e] = pack_bf16x2(d0, d1);
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 d4 = dv4[8 * ch + q4];
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int e = 4 * q4 + 2 * hh;  // within the 32-column chunk
+            const uint64_t dd = hh ? f2_pack(d4.z, d4.w) : f2_pack(d4.x, d4.y);
+            const uint64_t ds2 =
+                f2_mul(pf[16 * ch + (e >> 1)], f2_sub(f2_pack(__uint_as_float(dpr[e]), __uint_as_float(dpr[e + 1])), dd));
+            float d0, d1;
+            f2_unpack(ds2, d0, d1);
+            w[e >> 1] = pack_bf16x2(d0, d1);
+          }
         }
         // 128-byte swizzle: 16-byte unit u of row r lives at unit (u ^ (r & 7))
 #pragma unroll
@@ -379,28 +426,21 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
   } else if (warp < 12) {
     // ------------------------------------------------------------ dQ drain
     // Warp w owns query rows [32 w, 32 w + 32) of the partial.  Columns go in
-    // 64-wide passes through an 8 KB slice of the dS buffer (free once the dK
-    // and dQ MMAs that read dS are done, i.e. once the partial is ready), laid
-    // out as two 32-column TMA boxes with 128-byte swizzle; one lane then
-    // issues the TMA reduce-adds into the fp32 accumulator.
+    // 64-wide passes through an 8 KB staging slice (at d = 128 in the dO
+    // buffer of this step, which dV and dP have finished reading once the
+    // partial is ready), laid out as two 32-column TMA boxes with 128-byte
+    // swizzle; one lane then issues the TMA reduce-adds into the fp32
+    // accumulator.  The slice is handed back (bar_doempty) once the TMA
+    // engine has read it.
     const int wq = warp & 3;
     const uint32_t tQ = tmem + (static_cast<uint32_t>(wq * 32) << 16) + C::kColDQ;
-    uint8_t* stage = sDS + wq * 8192;
-    uint8_t* my_row = stage + lane * 128;
     const uint32_t swz = static_cast<uint32_t>(lane & 7);
-    auto stage_pass = [&](const uint32_t (&a)[32], const uint32_t (&b)[32]) {
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        *reinterpret_cast<uint4*>(my_row + ((u ^ swz) << 4)) = make_uint4(a[4 * u], a[4 * u + 1], a[4 * u + 2], a[4 * u + 3]);
-        *reinterpret_cast<uint4*>(my_row + 4096 + ((u ^ swz) << 4)) =
-            make_uint4(b[4 * u], b[4 * u + 1], b[4 * u + 2], b[4 * u + 3]);
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-    };
     for (int it = 0; it < n; ++it) {
+      const int st = it & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(bar_dqfull, it & 1, abort_flag, tmo, 230))) break;
       tc_fence_after();
+      uint8_t* stage = (D == 128 ? sDO + st * TILE : smem + C::kOffStage) + wq * 8192;
+      uint8_t* my_row = stage + lane * 128;
       const int grow = bh * p.Np + (i0 + it) * 128 + wq * 32;  // first accumulator row of this warp
       uint32_t a[32], b[32];
       tmem_ld32(tQ, a);
@@ -410,7 +450,14 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
         tc_fence_before();
         mbar_arrive(bar_dqfree);
       }
-      stage_pass(a, b);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        *reinterpret_cast<uint4*>(my_row + ((u ^ swz) << 4)) = make_uint4(a[4 * u], a[4 * u + 1], a[4 * u + 2], a[4 * u + 3]);
+        *reinterpret_cast<uint4*>(my_row + 4096 + ((u ^ swz) << 4)) =
+            make_uint4(b[4 * u], b[4 * u + 1], b[4 * u + 2], b[4 * u + 3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
       if (lane == 0) {
         tma_reduce_add_2d(stage, &p.tm_dq, 0, grow);
         tma_reduce_add_2d(stage + 4096, &p.tm_dq, 32, grow);
@@ -424,7 +471,15 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
         mbar_arrive(bar_dqfree);
         if (lane == 0) bulk_wait_group_read0();  // the first pass has left shared memory
         __syncwarp();
-        stage_pass(a, b);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          *reinterpret_cast<uint4*>(my_row + ((u ^ swz) << 4)) =
+              make_uint4(a[4 * u], a[4 * u + 1], a[4 * u + 2], a[4 * u + 3]);
+          *reinterpret_cast<uint4*>(my_row + 4096 + ((u ^ swz) << 4)) =
+              make_uint4(b[4 * u], b[4 * u + 1], b[4 * u + 2], b[4 * u + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
         if (lane == 0) {
           tma_reduce_add_2d(stage, &p.tm_dq, 64, grow);
           tma_reduce_add_2d(stage + 4096, &p.tm_dq, 96, grow);
@@ -433,7 +488,7 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
       }
       if (lane == 0) {
         bulk_wait_group_read0();
-        mbar_arrive(bar_dsfree);  // the compute warps may write the next dS
+        mbar_arrive(&bar_doempty[st]);  // the producer may load the next dO into this stage
       }
       __syncwarp();
     }
