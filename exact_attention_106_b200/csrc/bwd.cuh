@@ -289,18 +289,25 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
     // ------------------------------------------------------------ compute
     const int h = warp >> 2;  // query-column half
     const int wq = warp & 3;
-    const int r = wq * 32 + lane;  // key row in the tile
-    const int key = j * 128 + r;
+    const int key = j * 128 + wq * 32 + lane;  // epilogue: this thread's key row
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    // Each half reads its 64 score columns and writes its 64 bf16 probabilities
-    // (32 columns) over the first half of those same columns, so the two
-    // halves never touch each other's columns.
+    // Scores, dP and P are read and written in the 16-lane fragment layout:
+    // thread t holds key rows 32wq + 16b + 8rr + t/4 (b, rr in {0, 1}) and, in
+    // each 8-column group g of this half, the query pair 64h + 8g + 2(t%4) + {0, 1}.
+    // A thread thus needs only 16 of the 64 LSE and D values of its half, and
+    // each pair of them is one packed operand.
+    const int g4 = lane >> 2, t4 = lane & 3;
     const uint32_t tS = tmem + lane_off + C::kColS + 64 * h;
-    const uint32_t tP = tS;
     const uint32_t tDP = tmem + lane_off + C::kColDP + 64 * h;
     const float c = p.scale_log2;
-    const bool key_ok = key < N;
-    uint8_t* ds_row = sDS + h * 16384 + r * 128;
+    int pad = 0;  // bit 2b+rr: that key row is padding
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (j * 128 + 32 * wq + 8 * q + g4 >= N) pad |= 1 << q;
+    // dS tile: K-major, row = key, 128-byte swizzle (16-byte unit u of row k at
+    // unit u ^ (k & 7)); stmatrix row address of this lane for block b, group g
+    const uint32_t ds_lane = smem_u32(sDS) + h * 16384 + (32 * wq + (lane & 15)) * 128;
+    const uint32_t ds_sw = lane & 7;
     bool ok = true;
     for (int it = 0; it < n; ++it) {
       const int st = it & 1;
@@ -309,53 +316,69 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
         break;
       }
       tc_fence_after();
-      uint32_t sr[64];
-      tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      uint32_t sr[2][32];
+      tmem_ld16x256_x8(tS, sr[0]);
+      tmem_ld16x256_x8(tS + (16u << 16), sr[1]);
       tmem_wait_ld();
-      const float4* lse4 = reinterpret_cast<const float4*>(sVec + st * 256 + 64 * h);
-      const float4* dv4 = reinterpret_cast<const float4*>(sVec + st * 256 + 128 + 64 * h);
+      const float2* lse2 = reinterpret_cast<const float2*>(sVec + st * 256 + 64 * h + 2 * t4);
+      const float2* dv2 = reinterpret_cast<const float2*>(sVec + st * 256 + 128 + 64 * h + 2 * t4);
       const bool diag = p.causal && (it == 0);
-      // P^T = exp2(S^T c - LSE log2 e), in packed pairs; kEmuPairs of every 8
+      // P^T = exp2(S^T c - LSE log2 e) in packed pairs; kEmuPairs of every 8
       // pairs on the FMA pipe (ex2_fma2), the rest on the special-function unit
       const uint64_t c2 = f2_pack(c, c);
-      uint64_t pf[32];
+      uint64_t pf[2][16];  // [b][2g + rr]
 #pragma unroll
-      for (int q4 = 0; q4 < 16; ++q4) {
-        const float4 l4 = lse4[q4];
+      for (int g = 0; g < 8; ++g) {
+        const float2 l2 = lse2[4 * g];
+        const uint64_t nl = f2_pack(-l2.x, -l2.y);
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int e = 4 * q4 + 2 * hh;
-          const uint64_t nl = hh ? f2_pack(-l4.z, -l4.w) : f2_pack(-l4.x, -l4.y);
-          const uint64_t x = f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), c2, nl);
-          if (((e >> 1) & 7) >= 8 - kEmuPairs) {
-            pf[e >> 1] = ex2_fma2(x);
-          } else {
-            float x0, x1;
-            f2_unpack(x, x0, x1);
-            pf[e >> 1] = f2_pack(ex2(x0), ex2(x1));
+        for (int b = 0; b < 2; ++b) {
+#pragma unroll
+          for (int rr = 0; rr < 2; ++rr) {
+            const uint64_t x =
+                f2_fma(f2_pack(__uint_as_float(sr[b][4 * g + 2 * rr]), __uint_as_float(sr[b][4 * g + 2 * rr + 1])), c2, nl);
+            if (((2 * g + rr) & 7) >= 8 - kEmuPairs) {
+              pf[b][2 * g + rr] = ex2_fma2(x);
+            } else {
+              float x0, x1;
+              f2_unpack(x, x0, x1);
+              pf[b][2 * g + rr] = f2_pack(ex2(x0), ex2(x1));
+            }
           }
         }
       }
-      if (!key_ok || diag) {  // the key is padding, or the tile is on the diagonal
+      if (pad != 0 || diag) {  // padding key rows, or the tile is on the diagonal
 #pragma unroll
-        for (int e2 = 0; e2 < 32; ++e2) {
-          float p0, p1;
-          f2_unpack(pf[e2], p0, p1);
-          if (!key_ok || (diag && r > 64 * h + 2 * e2)) p0 = 0.f;
-          if (!key_ok || (diag && r > 64 * h + 2 * e2 + 1)) p1 = 0.f;
-          pf[e2] = f2_pack(p0, p1);
+        for (int b = 0; b < 2; ++b) {
+#pragma unroll
+          for (int rr = 0; rr < 2; ++rr) {
+            const int k = 32 * wq + 16 * b + 8 * rr + g4;
+            const bool dead = (pad >> (2 * b + rr)) & 1;
+#pragma unroll
+            for (int g = 0; g < 8; ++g) {
+              const int q = 64 * h + 8 * g + 2 * t4;
+              float p0, p1;
+              f2_unpack(pf[b][2 * g + rr], p0, p1);
+              if (dead || (diag && k > q)) p0 = 0.f;
+              if (dead || (diag && k > q + 1)) p1 = 0.f;
+              pf[b][2 * g + rr] = f2_pack(p0, p1);
+            }
+          }
         }
       }
-      uint32_t pk[32];
+      // bf16 P^T over the first 32 columns of this half's scores: query pair
+      // 2m, 2m+1 of the half in column m (m = 4g + t%4)
 #pragma unroll
-      for (int e2 = 0; e2 < 32; ++e2) {
-        float p0, p1;
-        f2_unpack(pf[e2], p0, p1);
-        pk[e2] = pack_bf16x2(p0, p1);
+      for (int b = 0; b < 2; ++b) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float p0, p1;
+          f2_unpack(pf[b][e], p0, p1);
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16x128_x8(tS + (static_cast<uint32_t>(16 * b) << 16), pk);
       }
-      tmem_st16(tP, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
-      tmem_st16(tP + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_p);
@@ -370,31 +393,27 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
       }
       tc_fence_after();
 #pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
+      for (int b = 0; b < 2; ++b) {
         uint32_t dpr[32];
-        tmem_ld32(tDP + 32 * ch, dpr);
+        tmem_ld16x256_x8(tDP + (static_cast<uint32_t>(16 * b) << 16), dpr);
         tmem_wait_ld();
-        uint32_t w[16];
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          const float4 d4 = dv4[8 * ch + q4];
+        for (int g = 0; g < 8; ++g) {
+          const float2 d2 = dv2[4 * g];
+          const uint64_t dd = f2_pack(d2.x, d2.y);
+          uint32_t w[2];
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int e = 4 * q4 + 2 * hh;  // within the 32-column chunk
-            const uint64_t dd = hh ? f2_pack(d4.z, d4.w) : f2_pack(d4.x, d4.y);
-            const uint64_t ds2 =
-                f2_mul(pf[16 * ch + (e >> 1)], f2_sub(f2_pack(__uint_as_float(dpr[e]), __uint_as_float(dpr[e + 1])), dd));
+          for (int rr = 0; rr < 2; ++rr) {
+            const uint64_t ds2 = f2_mul(pf[b][2 * g + rr],
+                                        f2_sub(f2_pack(__uint_as_float(dpr[4 * g + 2 * rr]),
+                                                       __uint_as_float(dpr[4 * g + 2 * rr + 1])),
+                                               dd));
             float d0, d1;
             f2_unpack(ds2, d0, d1);
-            w[e >> 1] = pack_bf16x2(d0, d1);
+            w[rr] = pack_bf16x2(d0, d1);
           }
-        }
-        // 128-byte swizzle: 16-byte unit u of row r lives at unit (u ^ (r & 7))
-#pragma unroll
-        for (int u4 = 0; u4 < 4; ++u4) {
-          const int u = 4 * ch + u4;
-          *reinterpret_cast<uint4*>(ds_row + ((u ^ (r & 7)) << 4)) =
-              make_uint4(w[4 * u4], w[4 * u4 + 1], w[4 * u4 + 2], w[4 * u4 + 3]);
+          // rows 32wq + 16b + (lane & 15): 8x8 matrices rr = 0, 1 of column group g
+          stmatrix_x2(ds_lane + 16 * b * 128 + ((g ^ ds_sw) << 4), w[0], w[1]);
         }
       }
       fence_proxy_async_smem();
@@ -404,6 +423,7 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
     // epilogue: half 0 writes dK (times scale), half 1 writes dV
     if (ok && __all_sync(0xffffffffu, mbar_wait(bar_final, 0, abort_flag, tmo, 223))) {
       tc_fence_after();
+      const bool key_ok = key < N;
       const uint32_t tAcc = tmem + lane_off + (h == 0 ? C::kColDK : C::kColDV);
       const float mul = (h == 0) ? p.scale : 1.0f;
       __nv_bfloat16* out = (h == 0 ? p.dk : p.dv) + (static_cast<size_t>(bh) * N + key) * D;
