@@ -382,6 +382,9 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_p);
+      float2 dvv[8];  // this thread's D pairs, read while dP^T is being computed
+#pragma unroll
+      for (int g = 0; g < 8; ++g) dvv[g] = dv2[4 * g];
 
       if (!__all_sync(0xffffffffu, mbar_wait(bar_dp, it & 1, abort_flag, tmo, 221))) {
         ok = false;
@@ -399,8 +402,7 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
         tmem_wait_ld();
 #pragma unroll
         for (int g = 0; g < 8; ++g) {
-          const float2 d2 = dv2[4 * g];
-          const uint64_t dd = f2_pack(d2.x, d2.y);
+          const uint64_t dd = f2_pack(dvv[g].x, dvv[g].y);
           uint32_t w[2];
 #pragma unroll
           for (int rr = 0; rr < 2; ++rr) {
