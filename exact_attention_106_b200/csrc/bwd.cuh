@@ -53,8 +53,21 @@ struct BwdParams {
 template <int D>
 struct BwdCfg {
   // warps 0..3: compute, query columns 0..63; warps 4..7: columns 64..127;
-  // warps 8..11: dQ drain; warp 12: TMA producer; warp 13: MMA issuer.
-  static constexpr int kThreads = 448;
+  // warps 8..11: dQ drain; warp 12: TMA producer; warp 13: MMA issuer;
+  // warps 14, 15: idle (they complete the last warpgroup).
+  static constexpr int kThreads = 512;
+  // Registers per thread: the launch gives every thread R (the compiled count,
+  // at most 65536 / 512 = 128).  Warpgroup 3 (producer, MMA, idle) drops to
+  // kRegsSide and the drain warpgroup rises to kRegsDrain, so that it can hold
+  // a whole 128-column dQ partial.  This fits if kRegsDrain - R <= R - kRegsSide,
+  // i.e. R >= kRegsMin; the host refuses to launch a build with fewer.
+  static constexpr int kRegsDrain = 168;
+  static constexpr int kRegsSide = 64;
+  static constexpr int kRegsMin = (kRegsDrain + kRegsSide + 1) / 2;
+  static constexpr int kRegsMax = 65536 / kThreads;
+  static_assert(kRegsMin <= kRegsMax, "register split cannot fit");
+  // per sub-partition: one warp of each warpgroup
+  static_assert(2 * kRegsMax + kRegsDrain + kRegsSide <= 512, "sub-partition register file");
   static constexpr uint32_t kTile = 128u * D * 2u;
   static constexpr int kChunks = D / 64;
   static constexpr uint32_t kOffK = 0;
@@ -90,7 +103,7 @@ __device__ __forceinline__ void bwd_issue_t(uint32_t d_tmem, SmemDesc dKm, uint3
 }
 
 template <int D>
-__global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant__ BwdParams p) {
+__global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant__ BwdParams p) {
   using C = BwdCfg<D>;
   constexpr int kProducerWarp = 12;
   constexpr int kMmaWarp = 13;
@@ -165,6 +178,8 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
   const uint32_t tmem = *tmem_slot;
   const uint64_t tmo = p.timeout_ns;
 
+  if (warp >= 12) {
+  setmaxnreg_dec<C::kRegsSide>();
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -285,6 +300,7 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
       drain_wait(bar_drain, 0, 219);
     }
     __syncwarp();
+  }
   } else if (warp < 8) {
     // ------------------------------------------------------------ compute
     const int h = warp >> 2;  // query-column half
@@ -445,7 +461,8 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
         }
       }
     }
-  } else if (warp < 12) {
+  } else {
+    setmaxnreg_inc<C::kRegsDrain>();
     // ------------------------------------------------------------ dQ drain
     // Warp w owns query rows [32 w, 32 w + 32) of the partial.  Columns go in
     // 64-wide passes through an 8 KB staging slice (at d = 128 in the dO
@@ -464,14 +481,17 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
       uint8_t* stage = (D == 128 ? sDO + st * TILE : smem + C::kOffStage) + wq * 8192;
       uint8_t* my_row = stage + lane * 128;
       const int grow = bh * p.Np + (i0 + it) * 128 + wq * 32;  // first accumulator row of this warp
-      uint32_t a[32], b[32];
+      uint32_t a[32], b[32], a2[32], b2[32];
       tmem_ld32(tQ, a);
       tmem_ld32(tQ + 32, b);
-      tmem_wait_ld();
-      if (D == 64) {  // every read of this partial is complete: hand the columns back
-        tc_fence_before();
-        mbar_arrive(bar_dqfree);
+      if (D == 128) {
+        tmem_ld32(tQ + 64, a2);
+        tmem_ld32(tQ + 96, b2);
       }
+      tmem_wait_ld();
+      // every read of this partial is complete: hand the columns back
+      tc_fence_before();
+      mbar_arrive(bar_dqfree);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         *reinterpret_cast<uint4*>(my_row + ((u ^ swz) << 4)) = make_uint4(a[4 * u], a[4 * u + 1], a[4 * u + 2], a[4 * u + 3]);
@@ -486,19 +506,14 @@ __global__ void __launch_bounds__(448, 1) attn_bwd_kernel(const __grid_constant_
         bulk_commit_group();
       }
       if (D == 128) {
-        tmem_ld32(tQ + 64, a);
-        tmem_ld32(tQ + 96, b);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(bar_dqfree);
         if (lane == 0) bulk_wait_group_read0();  // the first pass has left shared memory
         __syncwarp();
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           *reinterpret_cast<uint4*>(my_row + ((u ^ swz) << 4)) =
-              make_uint4(a[4 * u], a[4 * u + 1], a[4 * u + 2], a[4 * u + 3]);
+              make_uint4(a2[4 * u], a2[4 * u + 1], a2[4 * u + 2], a2[4 * u + 3]);
           *reinterpret_cast<uint4*>(my_row + 4096 + ((u ^ swz) << 4)) =
-              make_uint4(b[4 * u], b[4 * u + 1], b[4 * u + 2], b[4 * u + 3]);
+              make_uint4(b2[4 * u], b2[4 * u + 1], b2[4 * u + 2], b2[4 * u + 3]);
         }
         fence_proxy_async_smem();
         __syncwarp();

@@ -131,6 +131,21 @@ bool ensure_smem_attr(K kernel, int dev, std::atomic<int>* flags, int bytes) {
   return true;
 }
 
+// The backward kernel rebalances registers between warpgroups (setmaxnreg);
+// the split is only safe for a compiled register count in [kRegsMin, kRegsMax],
+// so a build outside that range is refused before its first launch.
+template <int D>
+bool bwd_regs_ok(int dev, std::atomic<int>* flags) {
+  if (flags[dev].load(std::memory_order_acquire)) return true;
+  cudaFuncAttributes a{};
+  if (cudaFuncGetAttributes(&a, exattn::attn_bwd_kernel<D>) != cudaSuccess) return false;
+  if (a.numRegs < exattn::BwdCfg<D>::kRegsMin || a.numRegs > exattn::BwdCfg<D>::kRegsMax) return false;
+  flags[dev].store(1, std::memory_order_release);
+  return true;
+}
+std::atomic<int> g_bwd64_regs[kMaxDevices];
+std::atomic<int> g_bwd128_regs[kMaxDevices];
+
 std::atomic<int> g_fwd64_attr[kMaxDevices];
 std::atomic<int> g_fwd128_attr[kMaxDevices];
 std::atomic<int> g_bwd64_attr[kMaxDevices];
@@ -258,10 +273,12 @@ int attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, v
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 64) {
     constexpr int smem = exattn::BwdCfg<64>::kSmem;
+    if (!bwd_regs_ok<64>(dev, g_bwd64_regs)) return ATTN_ERR_LAUNCH;
     if (!ensure_smem_attr(exattn::attn_bwd_kernel<64>, dev, g_bwd64_attr, smem)) return ATTN_ERR_LAUNCH;
     exattn::attn_bwd_kernel<64><<<grid, exattn::BwdCfg<64>::kThreads, smem, s>>>(p);
   } else {
     constexpr int smem = exattn::BwdCfg<128>::kSmem;
+    if (!bwd_regs_ok<128>(dev, g_bwd128_regs)) return ATTN_ERR_LAUNCH;
     if (!ensure_smem_attr(exattn::attn_bwd_kernel<128>, dev, g_bwd128_attr, smem)) return ATTN_ERR_LAUNCH;
     exattn::attn_bwd_kernel<128><<<grid, exattn::BwdCfg<128>::kThreads, smem, s>>>(p);
   }

@@ -270,6 +270,22 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
+// Register rebalancing between warpgroups (sm_90a+).  Every warp of a
+// warpgroup executes the same instruction.  .inc draws only on registers that
+// other warpgroups of the CTA released with .dec, so a split is safe only if
+// the increases sum to no more than the decreases (checked on the host
+// against the compiled register count before launch).
+template <uint32_t R>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  static_assert(R % 8 == 0 && R >= 24 && R <= 256, "setmaxnreg operand");
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <uint32_t R>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  static_assert(R % 8 == 0 && R >= 24 && R <= 256, "setmaxnreg operand");
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+}
+
 // 16-lane fragment shapes (the lane field of taddr selects the first of the 16
 // lanes).  16x256b.x8: thread t holds, for column group g = 0..7, the four
 // words r[4g..4g+3] = (lane t/4, col 8g+2(t%4)), (lane t/4, col 8g+2(t%4)+1),
