@@ -53,8 +53,9 @@ struct BwdParams {
 template <int D>
 struct BwdCfg {
   // warps 0..3: compute, query columns 0..63; warps 4..7: columns 64..127;
-  // warps 8..11: dQ drain; warp 12: TMA producer; warp 13: MMA issuer;
-  // warps 14, 15: idle (they complete the last warpgroup).
+  // warps 8..11: dQ drain; warp 12: TMA producer; warp 13: MMA issuer of
+  // the products that follow the scores (S^T, dP^T, dV); warp 14: MMA issuer
+  // of the products of dS (dQ, dK); warp 15: idle (completes the warpgroup).
   static constexpr int kThreads = 512;
   // Registers per thread: the launch gives every thread R (the compiled count,
   // at most 65536 / 512 = 128).  Warpgroup 3 (producer, MMA, idle) drops to
@@ -106,7 +107,8 @@ template <int D>
 __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant__ BwdParams p) {
   using C = BwdCfg<D>;
   constexpr int kProducerWarp = 12;
-  constexpr int kMmaWarp = 13;
+  constexpr int kMmaWarp = 13;   // also allocates TMEM
+  constexpr int kMmaWarp2 = 14;
   constexpr uint32_t TILE = C::kTile;
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {
@@ -132,9 +134,10 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
   uint64_t* bar_dsfree = bars + 13;  // dS consumed by the dQ and dK MMAs
   uint64_t* bar_dqfull = bars + 14;  // dQ partial ready in TMEM
   uint64_t* bar_dqfree = bars + 15;  // dQ partial read out of TMEM (128 arrivals)
-  uint64_t* bar_final = bars + 16;   // all MMAs done
-  uint64_t* bar_drain = bars + 17;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
+  uint64_t* bar_final = bars + 16;   // all MMAs done (one commit from each issuer)
+  uint64_t* bar_drain = bars + 17;   // both issuers' MMAs done (2 commits)
+  uint64_t* bar_dvdone = bars + 18;  // dV_i done: dO_i is read (issuer commit)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -163,8 +166,9 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
     mbar_init(bar_dsfree, 1);
     mbar_init(bar_dqfull, 1);
     mbar_init(bar_dqfree, 128);
-    mbar_init(bar_final, 1);
-    mbar_init(bar_drain, 1);
+    mbar_init(bar_final, 2);
+    mbar_init(bar_drain, 2);
+    mbar_init(bar_dvdone, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -225,8 +229,12 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       }
     }
     __syncwarp();
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == kMmaWarp || warp == kMmaWarp2) {
+    // ------------------------------------------------------------ MMA issuers
+    // Two threads issue MMAs into the one tensor pipe, each waiting only on
+    // its own inputs, so that one keeps the pipe busy while the other waits.
+    // A commit covers only its own thread's MMAs; every hand-off between
+    // the two goes through a barrier below.
     if (lane == 0) {
       constexpr uint32_t idesc_kv = idesc_bf16_f32(128, D, 0, 1);  // dV, dK: B = dO / Q MN-major
       constexpr uint32_t idesc_q = idesc_bf16_f32(128, D, 1, 1);   // dQ: A = dS MN-major, B = K MN-major
@@ -235,64 +243,73 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       const SmemDesc dKm = make_desc_sw128(smem_u32(smem), 16, 1024);
       const SmemDesc dMN = make_desc_sw128(smem_u32(smem), 16384, 1024);
       constexpr uint32_t oK = C::kOffK, oV = C::kOffV, oQ = C::kOffQ, oDO = C::kOffDO, oDS = C::kOffDS;
-      bool ok = mbar_wait(bar_kv, 0, abort_flag, tmo, 210) && mbar_wait(&bar_qfull[0], 0, abort_flag, tmo, 211) &&
-                mbar_wait(&bar_dofull[0], 0, abort_flag, tmo, 212);
-      if (ok) {
-        tc_fence_after();
-        bwd_issue_t<D>(tmem + C::kColS, dKm, oK, oQ);
-        tc_commit(bar_s);
-        bwd_issue_t<D>(tmem + C::kColDP, dKm, oV, oDO);
-        tc_commit(bar_dp);
-      }
-      for (int it = 0; it < n && ok; ++it) {
-        const int st = it & 1;
-        const int st1 = (it + 1) & 1;
-        const uint32_t ph1 = ((it + 1) >> 1) & 1;
-        // dV += P^T dO_i   (A = P^T from TMEM, K = 128 queries; queries 0..63
-        // sit in columns [0,32) of the score block, 64..127 in [64,96))
-        if (!mbar_wait(bar_p, it & 1, abort_flag, tmo, 213)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + C::kColDV, tmem + C::kColS + (kk >> 2) * 64 + (kk & 3) * 8,
-                 desc_at(dMN, oDO + st * TILE + kk * 2048), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
-        // next S^T as early as possible: the softmax of tile it+1 overlaps dQ, dK of tile it
-        if (it + 1 < n) {
-          if (!mbar_wait(&bar_qfull[st1], ph1, abort_flag, tmo, 214)) break;
+      if (warp == kMmaWarp) {
+        // S^T = K Q_i^T, dP^T = V dO_i^T, dV += P^T dO_i
+        bool ok = mbar_wait(bar_kv, 0, abort_flag, tmo, 210) && mbar_wait(&bar_qfull[0], 0, abort_flag, tmo, 211) &&
+                  mbar_wait(&bar_dofull[0], 0, abort_flag, tmo, 212);
+        if (ok) {
           tc_fence_after();
-          bwd_issue_t<D>(tmem + C::kColS, dKm, oK, oQ + st1 * TILE);
+          bwd_issue_t<D>(tmem + C::kColS, dKm, oK, oQ);
           tc_commit(bar_s);
-        }
-        if (!mbar_wait(bar_ds, it & 1, abort_flag, tmo, 215)) break;
-        tc_fence_after();
-        if (D != 128 && it > 0) {  // separate dQ columns: only the previous dQ must be drained
-          if (!mbar_wait(bar_dqfree, (it - 1) & 1, abort_flag, tmo, 216)) break;
-          tc_fence_after();
-        }
-        // dQ_i partial = dS K_j   (A = dS MN-major in smem, B = K_j MN-major),
-        // first, so that its drain overlaps dK
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + C::kColDQ, desc_at(dMN, oDS + kk * 2048), desc_at(dMN, oK + kk * 2048), idesc_q,
-                 kk > 0 ? 1u : 0u);
-        tc_commit(bar_dqfull);  // also: dV_i and dP_i, the readers of dO_i, are done
-        // dK += dS^T Q_i   (A = dS^T K-major in smem, B = Q_i MN-major)
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t offa = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(tmem + C::kColDK, desc_at(dKm, oDS + offa), desc_at(dMN, oQ + st * TILE + kk * 2048), idesc_kv,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(bar_dsfree);
-        tc_commit(&bar_qempty[st]);
-        if (it + 1 < n) {
-          if (D == 128) {  // dP^T(it+1) overwrites the dQ partial: wait until it is read out
-            if (!mbar_wait(bar_dqfree, it & 1, abort_flag, tmo, 217)) break;
-          }
-          if (!mbar_wait(&bar_dofull[st1], ph1, abort_flag, tmo, 218)) break;
-          tc_fence_after();
-          bwd_issue_t<D>(tmem + C::kColDP, dKm, oV, oDO + st1 * TILE);
+          bwd_issue_t<D>(tmem + C::kColDP, dKm, oV, oDO);
           tc_commit(bar_dp);
+        }
+        for (int it = 0; it < n && ok; ++it) {
+          const int st = it & 1;
+          const int st1 = (it + 1) & 1;
+          const uint32_t ph1 = ((it + 1) >> 1) & 1;
+          // dV += P^T dO_i   (A = P^T from TMEM, K = 128 queries; queries 0..63
+          // sit in columns [0,32) of the score block, 64..127 in [64,96))
+          if (!mbar_wait(bar_p, it & 1, abort_flag, tmo, 213)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + C::kColDV, tmem + C::kColS + (kk >> 2) * 64 + (kk & 3) * 8,
+                   desc_at(dMN, oDO + st * TILE + kk * 2048), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(bar_dvdone);  // also dP_i: both readers of dO_i are done
+          if (it + 1 < n) {
+            // next S^T as early as possible: its softmax overlaps dQ, dK of tile it
+            if (!mbar_wait(&bar_qfull[st1], ph1, abort_flag, tmo, 214)) break;
+            tc_fence_after();
+            bwd_issue_t<D>(tmem + C::kColS, dKm, oK, oQ + st1 * TILE);
+            tc_commit(bar_s);
+            // dP^T(it+1) overwrites dP^T(it), read once dS_i is written, and at
+            // d = 128 also the dQ partial, free once the drain has read it
+            if (!mbar_wait(bar_ds, it & 1, abort_flag, tmo, 215)) break;
+            if (D == 128 && !mbar_wait(bar_dqfree, it & 1, abort_flag, tmo, 217)) break;
+            if (!mbar_wait(&bar_dofull[st1], ph1, abort_flag, tmo, 218)) break;
+            tc_fence_after();
+            bwd_issue_t<D>(tmem + C::kColDP, dKm, oV, oDO + st1 * TILE);
+            tc_commit(bar_dp);
+          }
+        }
+      } else {
+        // dQ_i partial = dS K_j, dK += dS^T Q_i
+        bool ok = mbar_wait(bar_kv, 0, abort_flag, tmo, 224);
+        for (int it = 0; it < n && ok; ++it) {
+          const int st = it & 1;
+          if (!mbar_wait(bar_ds, it & 1, abort_flag, tmo, 225)) break;
+          tc_fence_after();
+          if (D != 128 && it > 0) {  // separate dQ columns: only the previous dQ must be drained
+            if (!mbar_wait(bar_dqfree, (it - 1) & 1, abort_flag, tmo, 216)) break;
+            tc_fence_after();
+          }
+          // dQ first (A = dS MN-major in smem, B = K_j MN-major), so that its
+          // drain overlaps dK
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + C::kColDQ, desc_at(dMN, oDS + kk * 2048), desc_at(dMN, oK + kk * 2048), idesc_q,
+                   kk > 0 ? 1u : 0u);
+          tc_commit(bar_dqfull);
+          // dK += dS^T Q_i   (A = dS^T K-major in smem, B = Q_i MN-major)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t offa = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_ss(tmem + C::kColDK, desc_at(dKm, oDS + offa), desc_at(dMN, oQ + st * TILE + kk * 2048),
+                   idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(bar_dsfree);
+          tc_commit(&bar_qempty[st]);
         }
       }
       tc_commit(bar_final);
@@ -492,6 +509,9 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       // every read of this partial is complete: hand the columns back
       tc_fence_before();
       mbar_arrive(bar_dqfree);
+      // dV_i and dP_i have read dO_i: its buffer may take the staging, and
+      // be handed back to the producer afterwards
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_dvdone, it & 1, abort_flag, tmo, 232))) break;
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         *reinterpret_cast<uint4*>(my_row + ((u ^ swz) << 4)) = make_uint4(a[4 * u], a[4 * u + 1], a[4 * u + 2], a[4 * u + 3]);
