@@ -251,17 +251,18 @@ def run_ours(args, rank, world, local_rank):
     max_ms = reduce_max(elapsed_ms, dev)
     flops_step = w.fwd_flops() + w.bwd_flops()
 
-    # e2e: pinned host buffers -> device -> fwd + bwd -> host, every step
+    # e2e: one C-ABI call per step on page-locked host buffers (attn_fwd_bwd_host:
+    # inputs copied in, fwd + bwd, results copied out, pipelined over head chunks)
     hq, hk, hv, hdo = (x.pin_memory() for x in (q, k, v, do))
     ho, hdq, hdk, hdv = (torch.empty(w.shape, dtype=torch.bfloat16).pin_memory() for _ in range(4))
     hlse = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+    del qd, kd, vd, dod, o, lse, dq, dk, dv, ws
+    torch.cuda.empty_cache()
+    hbuf = torch.empty(max(1, ex.host_buffer_bytes(B, H, N, d)), dtype=torch.uint8, device=dev)
 
     def e2e_step():
-        for h, dv_ in ((hq, qd), (hk, kd), (hv, vd), (hdo, dod)):
-            dv_.copy_(h, non_blocking=True)
-        step()
-        for dv_, h in ((o, ho), (lse, hlse), (dq, hdq), (dk, hdk), (dv, hdv)):
-            h.copy_(dv_, non_blocking=True)
+        ex.forward_backward_host(hq, hk, hv, hdo, (ho, hlse, hdq, hdk, hdv), causal=w.causal,
+                                 scale=w.softmax_scale, device=dev, dev_buffer=hbuf)
 
     e2e_steps = max(1, min(args.steps, 20))
     for _ in range(2):
@@ -274,6 +275,8 @@ def run_ours(args, rank, world, local_rank):
     e1.record(stream)
     barrier()
     e2e_ms = reduce_max(e0.elapsed_time(e1), dev)
+    if ex.device_status(dev) != 0:
+        raise RuntimeError("device status not clean after the end-to-end steps")
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hdo))
     d2h = sum(x.numel() * x.element_size() for x in (ho, hlse, hdq, hdk, hdv))
 

@@ -20,7 +20,8 @@ import torch
 
 from . import _lib
 
-__all__ = ["forward", "backward", "bwd_workspace_bytes", "device_status", "ExattnError"]
+__all__ = ["forward", "backward", "forward_backward_host", "bwd_workspace_bytes", "host_buffer_bytes",
+           "device_status", "ExattnError"]
 
 ExattnError = _lib.ExattnError
 
@@ -104,6 +105,37 @@ def bwd_stages(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool = False,
     _lib.check("attn_bwd_dq_convert", lib.attn_bwd_dq_convert(
         dq.data_ptr(), B, H, N, d, sc, workspace.data_ptr(), workspace.numel(), st))
     yield "dq_convert"
+
+
+def host_buffer_bytes(B: int, H: int, N: int, d: int, heads_per_chunk: int = 0) -> int:
+    return int(_lib.load().attn_fwd_bwd_host_buffer_bytes(B, H, N, d, heads_per_chunk))
+
+
+def forward_backward_host(q, k, v, do, out, causal: bool = False, scale: Optional[float] = None,
+                          device=None, dev_buffer: Optional[torch.Tensor] = None, heads_per_chunk: int = 0):
+    """Forward and backward over HOST tensors, copies included (attn_fwd_bwd_host).
+
+    q, k, v, do: CPU bf16 [B, H, N, d] (page-locked for the copies to overlap the
+    kernels); out = (o, lse, dq, dk, dv), CPU tensors written once the current
+    stream of ``device`` reaches the end of the call's work.
+    """
+    tensors = (q, k, v, do) + tuple(out)
+    o, lse, dq, dk, dv = out
+    B, H, N, d = q.shape
+    for t in (q, k, v, do, o, dq, dk, dv):
+        if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or tuple(t.shape) != (B, H, N, d):
+            raise ValueError("q, k, v, do, o, dq, dk, dv must be contiguous CPU bfloat16 [B, H, N, d]")
+    if lse.is_cuda or lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, H, N):
+        raise ValueError("lse must be contiguous CPU float32 [B, H, N]")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    need = host_buffer_bytes(B, H, N, d, heads_per_chunk)
+    buf = torch.empty(max(1, need), dtype=torch.uint8, device=dev) if dev_buffer is None else dev_buffer
+    with torch.cuda.device(dev):
+        _lib.check("attn_fwd_bwd_host", _lib.load().attn_fwd_bwd_host(
+            *(t.data_ptr() for t in tensors[:4]), o.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+            dv.data_ptr(), B, H, N, d, _scale(d, scale), int(causal), buf.data_ptr(), buf.numel(),
+            int(heads_per_chunk), _stream(dev)))
+    return out
 
 
 def device_status(device=None) -> int:

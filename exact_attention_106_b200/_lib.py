@@ -27,6 +27,9 @@ SIGNATURES = {
     "attn_bwd_dkdv": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _sz, _vp]),
     "attn_bwd_dq_convert": (_i, [_vp, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
     "attn_bwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp]),
+    "attn_fwd_bwd_host": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _sz, _i,
+                               _vp]),
+    "attn_fwd_bwd_host_buffer_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "attn_set_wait_timeout_ns": (None, [ctypes.c_ulonglong]),
     "attn_debug_inject_stall": (None, [_i]),
     "attn_get_device_status": (_i, [_vp]),

@@ -397,3 +397,159 @@ extern "C" int attn_bwd_noalloc(const void* q, const void* k, const void* v, con
   return attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, scratch,
                   static_cast<size_t>(EXATTN_NOALLOC_SCRATCH_BYTES), stream);
 }
+
+// ---------------------------------------------------------------------------
+// Forward + backward over host-resident tensors: attn_fwd_bwd_host().
+//
+// The (batch, head) pairs are split into chunks; chunk c uses buffer set
+// c % kHostStages of the caller's device buffer.  Per chunk, on three streams:
+//   copy-in stream:  [wait: set free] H2D q, k, v, dO      -> in_done[set]
+//   caller's stream: [wait: in_done] fwd -> fwd_done[set], bwd -> bwd_done[set]
+//   copy-out stream: [wait: fwd_done] D2H o, lse; [wait: bwd_done] D2H dq, dk,
+//                    dv -> free[set]
+// Events are recorded and waited on in host order, so each wait sees the
+// record of the same chunk.  Entry and exit are tied to the caller's stream.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int kHostStages = 2;
+
+struct HostPipe {
+  bool ready = false;
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, end = nullptr;
+  cudaEvent_t in_done[kHostStages] = {}, fwd_done[kHostStages] = {}, bwd_done[kHostStages] = {},
+              free_[kHostStages] = {};
+};
+
+std::mutex g_pipe_mu;  // guards g_pipe and serialises the enqueue sequences that use it
+HostPipe g_pipe[kMaxDevices];
+
+int pipe_for(int dev, HostPipe** out) {
+  HostPipe& hp = g_pipe[dev];
+  if (!hp.ready) {
+    const unsigned ef = cudaEventDisableTiming;
+    bool ok = cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.start, ef) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.end, ef) == cudaSuccess;
+    for (int s = 0; ok && s < kHostStages; ++s)
+      ok = cudaEventCreateWithFlags(&hp.in_done[s], ef) == cudaSuccess &&
+           cudaEventCreateWithFlags(&hp.fwd_done[s], ef) == cudaSuccess &&
+           cudaEventCreateWithFlags(&hp.bwd_done[s], ef) == cudaSuccess &&
+           cudaEventCreateWithFlags(&hp.free_[s], ef) == cudaSuccess;
+    if (!ok) return ATTN_ERR_LAUNCH;
+    hp.ready = true;
+  }
+  *out = &hp;
+  return ATTN_OK;
+}
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+int chunk_pairs(int BH, int heads_per_chunk) {
+  if (heads_per_chunk > 0) return heads_per_chunk < BH ? heads_per_chunk : BH;
+  return (BH + 7) / 8;
+}
+
+// one buffer set: q, k, v, dO, o, dq, dk, dv, lse, backward workspace
+size_t stage_bytes(int G, int N, int d) {
+  const size_t t = round256(static_cast<size_t>(G) * N * d * 2);
+  return 8 * t + round256(static_cast<size_t>(G) * N * 4) + round256(workspace_bytes(1, G, N, d));
+}
+
+struct Stage {
+  char *q, *k, *v, *dO, *o, *dq, *dk, *dv;
+  float* lse;
+  void* ws;
+  size_t ws_bytes;
+};
+
+Stage carve_stage(char* base, int G, int N, int d) {
+  const size_t t = round256(static_cast<size_t>(G) * N * d * 2);
+  Stage s;
+  char** slots[8] = {&s.q, &s.k, &s.v, &s.dO, &s.o, &s.dq, &s.dk, &s.dv};
+  for (int i = 0; i < 8; ++i) *slots[i] = base + i * t;
+  s.lse = reinterpret_cast<float*>(base + 8 * t);
+  s.ws = base + 8 * t + round256(static_cast<size_t>(G) * N * 4);
+  s.ws_bytes = workspace_bytes(1, G, N, d);
+  return s;
+}
+
+}  // namespace
+
+extern "C" size_t attn_fwd_bwd_host_buffer_bytes(int B, int H, int N, int d, int heads_per_chunk) {
+  if (check_sizes(B, H, N, d) != 0 || heads_per_chunk < 0) return 0;
+  const int BH = B * H;
+  const int G = chunk_pairs(BH, heads_per_chunk);
+  const int stages = (BH + G - 1) / G < kHostStages ? (BH + G - 1) / G : kHostStages;
+  return static_cast<size_t>(stages) * stage_bytes(G, N, d);
+}
+
+extern "C" int attn_fwd_bwd_host(const void* q, const void* k, const void* v, const void* dO, void* o, float* lse,
+                                 void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
+                                 void* dev_buf, size_t dev_buf_bytes, int heads_per_chunk, attn_stream_t stream) {
+  const int sz = check_sizes(B, H, N, d);
+  if (sz < 0 || !check_scale(scale) || heads_per_chunk < 0) return ATTN_ERR_INVALID;
+  if (sz == 1) return ATTN_OK;
+  if (!q || !k || !v || !dO || !o || !lse || !dq || !dk || !dv || !dev_buf) return ATTN_ERR_INVALID;
+  if ((reinterpret_cast<uintptr_t>(dev_buf) & 255u) != 0) return ATTN_ERR_INVALID;
+  if (dev_buf_bytes < attn_fwd_bwd_host_buffer_bytes(B, H, N, d, heads_per_chunk)) return ATTN_ERR_INVALID;
+  int dev = 0;
+  if (int st = check_device(&dev)) return st;
+
+  const int BH = B * H;
+  const int G = chunk_pairs(BH, heads_per_chunk);
+  const int nchunks = (BH + G - 1) / G;
+  const size_t sbytes = stage_bytes(G, N, d);
+  const size_t row = static_cast<size_t>(N) * d * 2;  // bytes of one (batch, head) of a bf16 tensor
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  HostPipe* hp = nullptr;
+  if (int st = pipe_for(dev, &hp)) return st;
+  auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+  if (!ok(cudaEventRecord(hp->start, cs)) || !ok(cudaStreamWaitEvent(hp->in, hp->start, 0)) ||
+      !ok(cudaStreamWaitEvent(hp->out, hp->start, 0)))
+    return ATTN_ERR_LAUNCH;
+  for (int c = 0; c < nchunks; ++c) {
+    const int s = c % kHostStages;
+    const int h0 = c * G;
+    const int g = (BH - h0) < G ? (BH - h0) : G;
+    const size_t off = static_cast<size_t>(h0) * row, bytes = static_cast<size_t>(g) * row;
+    const size_t loff = static_cast<size_t>(h0) * N, lbytes = static_cast<size_t>(g) * N * 4;
+    const Stage st = carve_stage(static_cast<char*>(dev_buf) + s * sbytes, G, N, d);
+    // copy in, once chunk c - kHostStages has left this buffer set
+    if (c >= kHostStages && !ok(cudaStreamWaitEvent(hp->in, hp->free_[s], 0))) return ATTN_ERR_LAUNCH;
+    const void* src[4] = {q, k, v, dO};
+    char* dst[4] = {st.q, st.k, st.v, st.dO};
+    for (int i = 0; i < 4; ++i)
+      if (!ok(cudaMemcpyAsync(dst[i], static_cast<const char*>(src[i]) + off, bytes, cudaMemcpyHostToDevice,
+                              hp->in)))
+        return ATTN_ERR_LAUNCH;
+    if (!ok(cudaEventRecord(hp->in_done[s], hp->in))) return ATTN_ERR_LAUNCH;
+    // kernels on the caller's stream
+    if (!ok(cudaStreamWaitEvent(cs, hp->in_done[s], 0))) return ATTN_ERR_LAUNCH;
+    if (int e = attn_fwd(st.q, st.k, st.v, st.o, st.lse, 1, g, N, d, scale, causal, stream)) return e;
+    if (!ok(cudaEventRecord(hp->fwd_done[s], cs))) return ATTN_ERR_LAUNCH;
+    if (int e = attn_bwd(st.q, st.k, st.v, st.o, st.lse, st.dO, st.dq, st.dk, st.dv, 1, g, N, d, scale, causal,
+                         st.ws, st.ws_bytes, stream))
+      return e;
+    if (!ok(cudaEventRecord(hp->bwd_done[s], cs))) return ATTN_ERR_LAUNCH;
+    // copy out: O and LSE as soon as the forward is done, the gradients after the backward
+    if (!ok(cudaStreamWaitEvent(hp->out, hp->fwd_done[s], 0)) ||
+        !ok(cudaMemcpyAsync(static_cast<char*>(o) + off, st.o, bytes, cudaMemcpyDeviceToHost, hp->out)) ||
+        !ok(cudaMemcpyAsync(lse + loff, st.lse, lbytes, cudaMemcpyDeviceToHost, hp->out)) ||
+        !ok(cudaStreamWaitEvent(hp->out, hp->bwd_done[s], 0)))
+      return ATTN_ERR_LAUNCH;
+    void* hdst[3] = {dq, dk, dv};
+    const char* dsrc[3] = {st.dq, st.dk, st.dv};
+    for (int i = 0; i < 3; ++i)
+      if (!ok(cudaMemcpyAsync(static_cast<char*>(hdst[i]) + off, dsrc[i], bytes, cudaMemcpyDeviceToHost, hp->out)))
+        return ATTN_ERR_LAUNCH;
+    if (!ok(cudaEventRecord(hp->free_[s], hp->out))) return ATTN_ERR_LAUNCH;
+  }
+  // the caller's stream waits for the last copies out
+  if (!ok(cudaEventRecord(hp->end, hp->out)) || !ok(cudaStreamWaitEvent(cs, hp->end, 0))) return ATTN_ERR_LAUNCH;
+  return ATTN_OK;
+}

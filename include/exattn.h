@@ -157,6 +157,42 @@ int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
                      int causal, attn_stream_t stream);
 
 /*
+ * One forward and backward pass over tensors that live in HOST memory: the
+ * copies to and from the device are part of the call.  (The pages have no
+ * counterpart: it strings attn_fwd and attn_bwd above together with the
+ * transfers, for callers whose data is not resident on the GPU.)
+ *
+ *   q, k, v, dO     host, [B, H, N, d] bf16, read
+ *   o, dq, dk, dv   host, [B, H, N, d] bf16, written (as attn_fwd / attn_bwd)
+ *   lse             host, [B, H, N] fp32, written
+ *   dev_buf         device memory of at least
+ *                   attn_fwd_bwd_host_buffer_bytes(B, H, N, d, heads_per_chunk)
+ *                   bytes, 256-byte aligned, owned by the caller and not used
+ *                   by anything else until the call's work on `stream` ends
+ *   heads_per_chunk (batch, head) pairs per pipeline chunk; 0 = B*H/8
+ *                   rounded up
+ *
+ * The (batch, head) pairs are independent, so the call splits them into
+ * chunks of heads_per_chunk consecutive pairs and pipelines the chunks over
+ * two buffer sets in dev_buf: while chunk c runs its kernels on `stream`, the
+ * inputs of chunk c+1 are copied in and the results of chunk c-1 copied out,
+ * on two internal streams of this library.  Like the calls above it only
+ * enqueues work: all of it completes before anything enqueued on `stream`
+ * after the call, and the host buffers must stay valid until then.  For the
+ * copies to overlap, the host buffers must be page-locked (cudaHostAlloc or
+ * cudaHostRegister); pageable buffers give the same results, slower.
+ *
+ * Returns ATTN_OK (also for empty problems), ATTN_ERR_INVALID (a bad size,
+ * scale or pointer, or dev_buf too small or misaligned), or ATTN_ERR_LAUNCH.
+ */
+int attn_fwd_bwd_host(const void* q, const void* k, const void* v, const void* dO, void* o, float* lse, void* dq,
+                      void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, void* dev_buf,
+                      size_t dev_buf_bytes, int heads_per_chunk, attn_stream_t stream);
+
+/* Device bytes attn_fwd_bwd_host() needs; 0 if the sizes are invalid or empty. */
+size_t attn_fwd_bwd_host_buffer_bytes(int B, int H, int N, int d, int heads_per_chunk);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word of
  * the current device: ATTN_OK, or ATTN_ERR_TIMEOUT if any kernel of this
  * library gave up waiting since the last call (ATTN_ERR_LAUNCH if the

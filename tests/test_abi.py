@@ -80,3 +80,33 @@ def test_bwd_rejects_small_workspace_and_misalignment(lib):
     assert lib.attn_bwd_dkdv(P, P, P, P, P, P, 1, 2, 300, 128, 0.1, 1, P, 0, None) == _lib.ATTN_ERR_INVALID
     assert lib.attn_bwd_dq_convert(P, 1, 2, 300, 64, 0.0, P, need, None) == _lib.ATTN_ERR_INVALID
     assert lib.attn_bwd(*([P] * 9), 0, 2, 300, 128, 0.1, 1, None, 0, None) == _lib.ATTN_OK
+
+
+def _stage_bytes(G, N, d):
+    r = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    np_ = (N + 127) // 128 * 128
+    return 8 * r(G * N * d * 2) + r(G * N * 4) + r(G * np_ * d * 4 + 2 * G * np_ * 4)
+
+
+def test_host_buffer_size(lib):
+    # 32 pairs, automatic chunks of 4 pairs, two buffer sets
+    assert lib.attn_fwd_bwd_host_buffer_bytes(1, 32, 16384, 128, 0) == 2 * _stage_bytes(4, 16384, 128)
+    # fewer chunks than buffer sets: one set
+    assert lib.attn_fwd_bwd_host_buffer_bytes(1, 3, 300, 64, 8) == _stage_bytes(3, 300, 64)
+    assert lib.attn_fwd_bwd_host_buffer_bytes(2, 3, 300, 64, 4) == 2 * _stage_bytes(4, 300, 64)
+    assert lib.attn_fwd_bwd_host_buffer_bytes(1, 1, 8, 80, 0) == 0
+    assert lib.attn_fwd_bwd_host_buffer_bytes(1, 2, 8, 64, -1) == 0
+
+
+def test_host_call_rejects_bad_arguments(lib):
+    need = lib.attn_fwd_bwd_host_buffer_bytes(1, 2, 300, 128, 1)
+    host = [P] * 9
+    good = [1, 2, 300, 128, 0.1, 1]
+    assert lib.attn_fwd_bwd_host(*host, *good, P, need - 1, 1, None) == _lib.ATTN_ERR_INVALID  # buffer too small
+    assert lib.attn_fwd_bwd_host(*host, *good, P + 16, need, 1, None) == _lib.ATTN_ERR_INVALID  # misaligned
+    assert lib.attn_fwd_bwd_host(*host, *good, None, need, 1, None) == _lib.ATTN_ERR_INVALID
+    assert lib.attn_fwd_bwd_host(*host, *good, P, need, -1, None) == _lib.ATTN_ERR_INVALID
+    assert lib.attn_fwd_bwd_host(None, *host[1:], *good, P, need, 1, None) == _lib.ATTN_ERR_INVALID
+    assert lib.attn_fwd_bwd_host(*host, 1, 2, 300, 96, 0.1, 1, P, need, 1, None) == _lib.ATTN_ERR_INVALID
+    assert lib.attn_fwd_bwd_host(*host, 1, 2, 300, 128, 0.0, 1, P, need, 1, None) == _lib.ATTN_ERR_INVALID
+    assert lib.attn_fwd_bwd_host(*host, 1, 0, 300, 128, 0.1, 1, None, 0, 0, None) == _lib.ATTN_OK  # empty
