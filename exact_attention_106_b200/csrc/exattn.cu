@@ -412,7 +412,10 @@ extern "C" int attn_bwd_noalloc(const void* q, const void* k, const void* v, con
 // ---------------------------------------------------------------------------
 namespace {
 
-constexpr int kHostStages = 2;
+// Three buffer sets: chunk c+1 is copied in while chunk c computes and chunk
+// c-1 is copied out, without waiting for the copy-out of c-1 (as two sets
+// would), so the two PCIe directions run independently.
+constexpr int kHostStages = 3;
 
 struct HostPipe {
   bool ready = false;

@@ -174,9 +174,9 @@ int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
  *
  * The (batch, head) pairs are independent, so the call splits them into
  * chunks of heads_per_chunk consecutive pairs and pipelines the chunks over
- * two buffer sets in dev_buf: while chunk c runs its kernels on `stream`, the
- * inputs of chunk c+1 are copied in and the results of chunk c-1 copied out,
- * on two internal streams of this library.  Like the calls above it only
+ * three buffer sets in dev_buf: while chunk c runs its kernels on `stream`,
+ * the inputs of chunk c+1 are copied in and the results of chunk c-1 copied
+ * out, on two internal streams of this library.  Like the calls above it only
  * enqueues work: all of it completes before anything enqueued on `stream`
  * after the call, and the host buffers must stay valid until then.  For the
  * copies to overlap, the host buffers must be page-locked (cudaHostAlloc or

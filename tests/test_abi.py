@@ -89,11 +89,12 @@ def _stage_bytes(G, N, d):
 
 
 def test_host_buffer_size(lib):
-    # 32 pairs, automatic chunks of 4 pairs, two buffer sets
-    assert lib.attn_fwd_bwd_host_buffer_bytes(1, 32, 16384, 128, 0) == 2 * _stage_bytes(4, 16384, 128)
-    # fewer chunks than buffer sets: one set
+    # 32 pairs, automatic chunks of 4 pairs, three buffer sets
+    assert lib.attn_fwd_bwd_host_buffer_bytes(1, 32, 16384, 128, 0) == 3 * _stage_bytes(4, 16384, 128)
+    # fewer chunks than buffer sets: one set per chunk
     assert lib.attn_fwd_bwd_host_buffer_bytes(1, 3, 300, 64, 8) == _stage_bytes(3, 300, 64)
     assert lib.attn_fwd_bwd_host_buffer_bytes(2, 3, 300, 64, 4) == 2 * _stage_bytes(4, 300, 64)
+    assert lib.attn_fwd_bwd_host_buffer_bytes(2, 3, 300, 64, 1) == 3 * _stage_bytes(1, 300, 64)
     assert lib.attn_fwd_bwd_host_buffer_bytes(1, 1, 8, 80, 0) == 0
     assert lib.attn_fwd_bwd_host_buffer_bytes(1, 2, 8, 64, -1) == 0
 
