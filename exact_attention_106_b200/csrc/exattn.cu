@@ -481,6 +481,12 @@ Stage carve_stage(char* base, int G, int N, int d) {
 
 }  // namespace
 
+namespace {
+int enqueue_host_chunks(HostPipe* hp, const void* q, const void* k, const void* v, const void* dO, void* o,
+                        float* lse, void* dq, void* dk, void* dv, int N, int d, float scale, int causal,
+                        char* dev_buf, int G, int nchunks, int BH, size_t sbytes, size_t row, attn_stream_t stream);
+}  // namespace
+
 extern "C" size_t attn_fwd_bwd_host_buffer_bytes(int B, int H, int N, int d, int heads_per_chunk) {
   if (check_sizes(B, H, N, d) != 0 || heads_per_chunk < 0) return 0;
   const int BH = B * H;
@@ -515,13 +521,30 @@ extern "C" int attn_fwd_bwd_host(const void* q, const void* k, const void* v, co
   if (!ok(cudaEventRecord(hp->start, cs)) || !ok(cudaStreamWaitEvent(hp->in, hp->start, 0)) ||
       !ok(cudaStreamWaitEvent(hp->out, hp->start, 0)))
     return ATTN_ERR_LAUNCH;
+  const int st = enqueue_host_chunks(hp, q, k, v, dO, o, lse, dq, dk, dv, N, d, scale, causal,
+                                     static_cast<char*>(dev_buf), G, nchunks, BH, sbytes, row, stream);
+  // The caller's stream waits for everything enqueued above, also after a
+  // failure part-way, so that no copy still runs once the caller may free or
+  // reuse its buffers.
+  const bool tied = ok(cudaEventRecord(hp->end, hp->in)) && ok(cudaStreamWaitEvent(cs, hp->end, 0)) &&
+                    ok(cudaEventRecord(hp->end, hp->out)) && ok(cudaStreamWaitEvent(cs, hp->end, 0));
+  if (st != ATTN_OK) return st;
+  return tied ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+namespace {
+int enqueue_host_chunks(HostPipe* hp, const void* q, const void* k, const void* v, const void* dO, void* o,
+                        float* lse, void* dq, void* dk, void* dv, int N, int d, float scale, int causal,
+                        char* dev_buf, int G, int nchunks, int BH, size_t sbytes, size_t row, attn_stream_t stream) {
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  auto ok = [](cudaError_t e) { return e == cudaSuccess; };
   for (int c = 0; c < nchunks; ++c) {
     const int s = c % kHostStages;
     const int h0 = c * G;
     const int g = (BH - h0) < G ? (BH - h0) : G;
     const size_t off = static_cast<size_t>(h0) * row, bytes = static_cast<size_t>(g) * row;
     const size_t loff = static_cast<size_t>(h0) * N, lbytes = static_cast<size_t>(g) * N * 4;
-    const Stage st = carve_stage(static_cast<char*>(dev_buf) + s * sbytes, G, N, d);
+    const Stage st = carve_stage(dev_buf + s * sbytes, G, N, d);
     // copy in, once chunk c - kHostStages has left this buffer set
     if (c >= kHostStages && !ok(cudaStreamWaitEvent(hp->in, hp->free_[s], 0))) return ATTN_ERR_LAUNCH;
     const void* src[4] = {q, k, v, dO};
@@ -552,7 +575,7 @@ extern "C" int attn_fwd_bwd_host(const void* q, const void* k, const void* v, co
         return ATTN_ERR_LAUNCH;
     if (!ok(cudaEventRecord(hp->free_[s], hp->out))) return ATTN_ERR_LAUNCH;
   }
-  // the caller's stream waits for the last copies out
-  if (!ok(cudaEventRecord(hp->end, hp->out)) || !ok(cudaStreamWaitEvent(cs, hp->end, 0))) return ATTN_ERR_LAUNCH;
   return ATTN_OK;
 }
+}  // namespace
+
