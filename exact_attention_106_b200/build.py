@@ -15,6 +15,8 @@ import sys
 PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG_DIR)
 LIB_PATH = os.path.join(PKG_DIR, "libexattn.so")
+# ptxas's per-kernel resource report of the last build (registers, spills)
+RESOURCES_PATH = os.path.join(PKG_DIR, "libexattn.resources.txt")
 SOURCES = [os.path.join(PKG_DIR, "csrc", f) for f in ("exattn.cu", "ptx.cuh", "fwd.cuh", "bwd.cuh")]
 HEADER = os.path.join(ROOT, "include", "exattn.h")
 
@@ -26,19 +28,16 @@ def nvcc_path() -> str:
     raise RuntimeError("nvcc not found: cannot build the exattn CUDA library")
 
 
-def build_command(out: str = LIB_PATH, verbose_ptxas: bool = False):
-    cmd = [
-        nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
-        "-Xcompiler", "-fPIC", "-shared", "-I", os.path.join(ROOT, "include"),
+def build_command(out: str = LIB_PATH):
+    return [
+        nvcc_path(), "-Xptxas", "-v", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3",
+        "-std=c++17", "-Xcompiler", "-fPIC", "-shared", "-I", os.path.join(ROOT, "include"),
         "-o", out, os.path.join(PKG_DIR, "csrc", "exattn.cu"),
     ]
-    if verbose_ptxas:
-        cmd[1:1] = ["-Xptxas", "-v"]
-    return cmd
 
 
 def is_stale(out: str = LIB_PATH) -> bool:
-    if not os.path.exists(out):
+    if not os.path.exists(out) or not os.path.exists(RESOURCES_PATH):
         return True
     t = os.path.getmtime(out)
     return any(os.path.getmtime(s) > t for s in SOURCES + [HEADER, __file__])
@@ -47,12 +46,16 @@ def is_stale(out: str = LIB_PATH) -> bool:
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     if force or is_stale():
         tmp = LIB_PATH + ".tmp"
-        proc = subprocess.run(build_command(tmp, verbose_ptxas), capture_output=True, text=True)
+        proc = subprocess.run(build_command(tmp), capture_output=True, text=True)
         if proc.returncode != 0:
             raise RuntimeError("nvcc failed:\n" + proc.stdout + proc.stderr)
         if verbose_ptxas:
             sys.stderr.write(proc.stderr)
+        report = [ln for ln in proc.stderr.splitlines() if "ptxas info" in ln or "bytes stack frame" in ln]
+        with open(RESOURCES_PATH + ".tmp", "w") as f:
+            f.write("\n".join(report) + "\n")
         os.replace(tmp, LIB_PATH)
+        os.replace(RESOURCES_PATH + ".tmp", RESOURCES_PATH)
     return LIB_PATH
 
 

@@ -1,0 +1,68 @@
+"""Compiled register counts that the kernels' launch configurations rely on,
+read from ptxas's resource report of the in-tree build (no GPU needed).
+
+* A CTA's warps are spread over the SM's four sub-partitions, each with a
+  16K-register file: warps_per_sub_partition * 32 * registers <= 16384, or the
+  launch fails.
+* The backward moves registers between warpgroups with setmaxnreg: the drain
+  warpgroup's increase must not exceed what the producer/MMA warpgroup frees,
+  or setmaxnreg.inc waits forever (the host refuses such a build at run time;
+  this catches it at build time).
+"""
+import math
+import os
+import re
+
+import pytest
+
+from exact_attention_106_b200 import build
+
+CSRC = os.path.join(build.PKG_DIR, "csrc")
+
+
+@pytest.fixture(scope="module")
+def registers():
+    build.build()
+    regs, cur = {}, None
+    for line in open(build.RESOURCES_PATH).read().splitlines():
+        m = re.search(r"Compiling entry function '(\w+)'", line)
+        if m:
+            cur = m.group(1)
+            continue
+        m = re.search(r"Used (\d+) registers", line)
+        if m and cur:
+            regs[cur] = int(m.group(1))
+            cur = None
+    return regs
+
+
+def _const(path, name):
+    m = re.search(r"static constexpr int %s = (\d+);" % name, open(os.path.join(CSRC, path)).read())
+    assert m, name
+    return int(m.group(1))
+
+
+def _kernel(regs, stem, d, params):
+    name = f"_ZN6exattn{len(stem)}{stem}ILi{d}EEEvNS_{len(params)}{params}E"
+    assert name in regs, sorted(regs)
+    return regs[name]
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_backward_register_split_fits(registers, d):
+    r = _kernel(registers, "attn_bwd_kernel", d, "BwdParams")
+    threads = _const("bwd.cuh", "kThreads")
+    drain, side = _const("bwd.cuh", "kRegsDrain"), _const("bwd.cuh", "kRegsSide")
+    # warpgroup 2 (drain) rises from r to `drain`, warpgroup 3 falls from r to `side`
+    assert drain - r <= r - side, (r, drain, side)
+    per_sub = math.ceil(threads // 32 / 4)
+    assert per_sub * 32 * r <= 16384, (r, per_sub)
+    # after the split, one warp of each warpgroup per sub-partition
+    assert 32 * (2 * r + drain + side) <= 16384
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_forward_fits_the_sub_partitions(registers, d):
+    r = _kernel(registers, "attn_fwd_kernel", d, "FwdParams")
+    per_sub = math.ceil(_const("fwd.cuh", "kThreads") // 32 / 4)
+    assert per_sub * 32 * r <= 16384, (r, per_sub)
