@@ -43,8 +43,23 @@ def _scale(d: int, scale: Optional[float]) -> float:
     return 1.0 / math.sqrt(d) if scale is None else float(scale)
 
 
-def forward(q, k, v, causal: bool = False, scale: Optional[float] = None, out=None, lse=None):
-    """O and per-row logsumexp of softmax(scale Q K^T) V."""
+def _check_status(fn: str, device) -> None:
+    """Synchronise and raise if a kernel of the library gave up on a bounded
+    wait (the results of that call are then undefined)."""
+    st = device_status(device)
+    if st != _lib.ATTN_OK:
+        raise ExattnError(fn, st)
+
+
+def forward(q, k, v, causal: bool = False, scale: Optional[float] = None, out=None, lse=None,
+            check: bool = False):
+    """O and per-row logsumexp of softmax(scale Q K^T) V.
+
+    The call only enqueues the kernel.  A kernel that gives up on one of its
+    bounded internal waits (about a second; it should never happen) leaves
+    undefined outputs and records ATTN_ERR_TIMEOUT, which ``device_status()``
+    reports; with ``check=True`` the call synchronises and raises ExattnError
+    in that case."""
     _check_qkv(q, k, v)
     B, H, N, d = q.shape
     o = torch.empty_like(q) if out is None else out
@@ -53,6 +68,8 @@ def forward(q, k, v, causal: bool = False, scale: Optional[float] = None, out=No
     _lib.check("attn_fwd", lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                                         lse_t.data_ptr(), B, H, N, d, _scale(d, scale), int(causal),
                                         _stream(q.device)))
+    if check:
+        _check_status("attn_fwd", q.device)
     return o, lse_t
 
 
@@ -67,8 +84,12 @@ def alloc_workspace(B: int, H: int, N: int, d: int, device) -> torch.Tensor:
 
 
 def backward(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] = None,
-             workspace: Optional[torch.Tensor] = None, out=None):
-    """dQ, dK, dV of sum(O * dO) for O = softmax(scale Q K^T) V."""
+             workspace: Optional[torch.Tensor] = None, out=None, check: bool = False):
+    """dQ, dK, dV of sum(O * dO) for O = softmax(scale Q K^T) V.
+
+    ``check=True`` synchronises and raises ExattnError if a kernel gave up on
+    a bounded wait (see ``forward``); otherwise such a failure is only seen
+    through ``device_status()``."""
     _check_qkv(q, k, v, o, do)
     B, H, N, d = q.shape
     if not (lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous() and lse.shape == (B, H, N)):
@@ -83,6 +104,8 @@ def backward(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] =
         q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
         dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, _scale(d, scale), int(causal),
         ws.data_ptr(), ws.numel(), _stream(q.device)))
+    if check:
+        _check_status("attn_bwd", q.device)
     return dq, dk, dv
 
 
@@ -117,7 +140,8 @@ def forward_backward_host(q, k, v, do, out, causal: bool = False, scale: Optiona
 
     q, k, v, do: CPU bf16 [B, H, N, d] (page-locked for the copies to overlap the
     kernels); out = (o, lse, dq, dk, dv), CPU tensors written once the current
-    stream of ``device`` reaches the end of the call's work.
+    stream of ``device`` reaches the end of the call's work.  As with
+    ``forward``, a kernel timeout is reported only by ``device_status()``.
     """
     tensors = (q, k, v, do) + tuple(out)
     o, lse, dq, dk, dv = out

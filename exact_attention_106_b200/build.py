@@ -28,10 +28,13 @@ def nvcc_path() -> str:
     raise RuntimeError("nvcc not found: cannot build the exattn CUDA library")
 
 
-def build_command(out: str = LIB_PATH):
+def build_command(out: str = LIB_PATH, cudart: str = "static"):
+    """nvcc command line for the library.  ``cudart="shared"`` links the CUDA
+    runtime dynamically instead (the tests use such a build to share one
+    runtime with a caller that resets the device)."""
     return [
         nvcc_path(), "-Xptxas", "-v", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3",
-        "-std=c++17", "-Xcompiler", "-fPIC", "-shared", "-I", os.path.join(ROOT, "include"),
+        "-std=c++17", "-Xcompiler", "-fPIC", "-shared", f"-cudart={cudart}", "-I", os.path.join(ROOT, "include"),
         "-o", out, os.path.join(PKG_DIR, "csrc", "exattn.cu"),
     ]
 

@@ -136,8 +136,12 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
   uint64_t* bar_dqfree = bars + 15;  // dQ partial read out of TMEM (128 arrivals)
   uint64_t* bar_final = bars + 16;   // all MMAs done (one commit from each issuer)
   uint64_t* bar_drain = bars + 17;   // both issuers' MMAs done (2 commits)
-  uint64_t* bar_dvdone = bars + 18;  // dV_i done: dO_i is read (issuer commit)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
+  // [2] dV_i done, so dO_i is read (issuer commit), one per dO stage: the
+  // drain of step i waits on stage i % 2, whose next phase needs dO_(i+2),
+  // which only loads after that drain has released the stage, so the
+  // barrier can never run two phases ahead of its waiter
+  uint64_t* bar_dvdone = bars + 18;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -168,7 +172,8 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
     mbar_init(bar_dqfree, 128);
     mbar_init(bar_final, 2);
     mbar_init(bar_drain, 2);
-    mbar_init(bar_dvdone, 1);
+    mbar_init(&bar_dvdone[0], 1);
+    mbar_init(&bar_dvdone[1], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -266,7 +271,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
           for (int kk = 0; kk < 8; ++kk)
             mma_ts(tmem + C::kColDV, tmem + C::kColS + (kk >> 2) * 64 + (kk & 3) * 8,
                    desc_at(dMN, oDO + st * TILE + kk * 2048), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
-          tc_commit(bar_dvdone);  // also dP_i: both readers of dO_i are done
+          tc_commit(&bar_dvdone[st]);  // also dP_i: both readers of dO_i are done
           if (it + 1 < n) {
             // next S^T as early as possible: its softmax overlaps dQ, dK of tile it
             if (!mbar_wait(&bar_qfull[st1], ph1, abort_flag, tmo, 214)) break;
@@ -511,7 +516,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       mbar_arrive(bar_dqfree);
       // dV_i and dP_i have read dO_i: its buffer may take the staging, and
       // be handed back to the producer afterwards
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_dvdone, it & 1, abort_flag, tmo, 232))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar_dvdone[st], (it >> 1) & 1, abort_flag, tmo, 232))) break;
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         *reinterpret_cast<uint4*>(my_row + ((u ^ swz) << 4)) = make_uint4(a[4 * u], a[4 * u + 1], a[4 * u + 2], a[4 * u + 3]);

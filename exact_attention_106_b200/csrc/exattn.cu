@@ -121,14 +121,12 @@ bool make_map_f32_dq(CUtensorMap* m, void* base, size_t rows, int d) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Per-device, per-kernel one-time opt-in to large dynamic shared memory.
+// Opt-in to large dynamic shared memory, set before every launch: the
+// attribute belongs to the loaded module, which a re-created context
+// (cudaDeviceReset) loads afresh.  It is a host-side call.
 template <typename K>
-bool ensure_smem_attr(K kernel, int dev, std::atomic<int>* flags, int bytes) {
-  if (flags[dev].load(std::memory_order_acquire)) return true;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
-    return false;
-  flags[dev].store(1, std::memory_order_release);
-  return true;
+bool ensure_smem_attr(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
 }
 
 // The backward kernel rebalances registers between warpgroups (setmaxnreg);
@@ -146,10 +144,6 @@ bool bwd_regs_ok(int dev, std::atomic<int>* flags) {
 std::atomic<int> g_bwd64_regs[kMaxDevices];
 std::atomic<int> g_bwd128_regs[kMaxDevices];
 
-std::atomic<int> g_fwd64_attr[kMaxDevices];
-std::atomic<int> g_fwd128_attr[kMaxDevices];
-std::atomic<int> g_bwd64_attr[kMaxDevices];
-std::atomic<int> g_bwd128_attr[kMaxDevices];
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH; }
 
@@ -198,11 +192,11 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 64) {
     constexpr int smem = exattn::FwdCfg<64>::kSmem;
-    if (!ensure_smem_attr(exattn::attn_fwd_kernel<64>, dev, g_fwd64_attr, smem)) return ATTN_ERR_LAUNCH;
+    if (!ensure_smem_attr(exattn::attn_fwd_kernel<64>, smem)) return ATTN_ERR_LAUNCH;
     exattn::attn_fwd_kernel<64><<<grid, exattn::FwdCfg<64>::kThreads, smem, s>>>(p);
   } else {
     constexpr int smem = exattn::FwdCfg<128>::kSmem;
-    if (!ensure_smem_attr(exattn::attn_fwd_kernel<128>, dev, g_fwd128_attr, smem)) return ATTN_ERR_LAUNCH;
+    if (!ensure_smem_attr(exattn::attn_fwd_kernel<128>, smem)) return ATTN_ERR_LAUNCH;
     exattn::attn_fwd_kernel<128><<<grid, exattn::FwdCfg<128>::kThreads, smem, s>>>(p);
   }
   return launch_status();
@@ -274,12 +268,12 @@ int attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, v
   if (d == 64) {
     constexpr int smem = exattn::BwdCfg<64>::kSmem;
     if (!bwd_regs_ok<64>(dev, g_bwd64_regs)) return ATTN_ERR_LAUNCH;
-    if (!ensure_smem_attr(exattn::attn_bwd_kernel<64>, dev, g_bwd64_attr, smem)) return ATTN_ERR_LAUNCH;
+    if (!ensure_smem_attr(exattn::attn_bwd_kernel<64>, smem)) return ATTN_ERR_LAUNCH;
     exattn::attn_bwd_kernel<64><<<grid, exattn::BwdCfg<64>::kThreads, smem, s>>>(p);
   } else {
     constexpr int smem = exattn::BwdCfg<128>::kSmem;
     if (!bwd_regs_ok<128>(dev, g_bwd128_regs)) return ATTN_ERR_LAUNCH;
-    if (!ensure_smem_attr(exattn::attn_bwd_kernel<128>, dev, g_bwd128_attr, smem)) return ATTN_ERR_LAUNCH;
+    if (!ensure_smem_attr(exattn::attn_bwd_kernel<128>, smem)) return ATTN_ERR_LAUNCH;
     exattn::attn_bwd_kernel<128><<<grid, exattn::BwdCfg<128>::kThreads, smem, s>>>(p);
   }
   return launch_status();
@@ -359,25 +353,22 @@ const char* attn_status_string(int status) {
 // vectors) lives in one file-scope __device__ array of
 // EXATTN_NOALLOC_SCRATCH_BYTES, which every GPU that loads this library holds
 // until the process exits.  In host code the array's name is only a host-side
-// stand-in, so its device address is fetched once per device with
-// cudaGetSymbolAddress (on the first call made with that device current) and
-// passed to the kernels.
+// stand-in, so its device address is fetched with cudaGetSymbolAddress, on
+// every call with the caller's device current, and passed to the kernels.
 // ---------------------------------------------------------------------------
 namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[EXATTN_NOALLOC_SCRATCH_BYTES];
 
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices];  // device address of g_noalloc_scratch, per device; guarded by g_noalloc_mu
-
-int noalloc_scratch_address(int dev, void** out) {
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return ATTN_ERR_LAUNCH;
-    g_noalloc_ptr[dev] = p;
-  }
-  *out = g_noalloc_ptr[dev];
+// The array's device address in the current device's context.  It is looked
+// up on every call rather than cached: after cudaDeviceReset (or any other
+// re-creation of the primary context) the module is loaded again and the
+// array may sit at a different address.  The lookup is a host-side table
+// read, no device work.
+int noalloc_scratch_address(void** out) {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return ATTN_ERR_LAUNCH;
+  *out = p;
   return ATTN_OK;
 }
 
@@ -393,7 +384,7 @@ extern "C" int attn_bwd_noalloc(const void* q, const void* k, const void* v, con
   int dev = 0;
   if (int st = check_device(&dev)) return st;
   void* scratch = nullptr;
-  if (int st = noalloc_scratch_address(dev, &scratch)) return st;
+  if (int st = noalloc_scratch_address(&scratch)) return st;
   return attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, scratch,
                   static_cast<size_t>(EXATTN_NOALLOC_SCRATCH_BYTES), stream);
 }

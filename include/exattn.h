@@ -143,8 +143,11 @@ int attn_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, const
  *    EXATTN_NOALLOC_SCRATCH_BYTES are rejected with ATTN_ERR_INVALID before
  *    anything runs: for d = 128 when B*H*ceil(N/128) > 1008, for d = 64
  *    when B*H*ceil(N/128) > 1985.
- *  - The first call on a device looks up the array's device address (with
- *    that device current); make that first call before any stream capture.
+ *  - Every call looks up the array's device address in the current device's
+ *    context (a host-side lookup, no device work), so a context that was
+ *    re-created, e.g. after cudaDeviceReset, is followed.  The first call on
+ *    a device may load the library's kernels into the context: make it
+ *    before any stream capture.
  *  - Every call on a device shares the one array.  Each call re-initialises
  *    the parts it reads, so leftover contents never leak into results, but
  *    calls that overlap on the GPU (other streams, other host threads) race

@@ -44,3 +44,24 @@ def test_wait_limit_runs_out_and_context_survives(cuda_device, d):
     got = run_cuda(q, k, v, do, True, scale)
     ref = oracle_ref(q, k, v, do, True, scale)
     check_all(got, ref, what=f"after timeout d={d}")
+
+
+def test_check_flag_raises_on_timeout(cuda_device):
+    """forward(check=True) / backward(check=True) turn a recorded wait timeout
+    into ExattnError instead of returning undefined outputs silently."""
+    lib = _lib.load()
+    g = torch.Generator().manual_seed(5)
+    q, k, v, do = (torch.randn((1, 2, 300, 128), generator=g).bfloat16().to(cuda_device) for _ in range(4))
+    o, lse = ex.forward(q, k, v, causal=True, check=True)  # clean run: no raise
+    lib.attn_set_wait_timeout_ns(20_000_000)
+    lib.attn_debug_inject_stall(1)
+    try:
+        with pytest.raises(ex.ExattnError) as e1:
+            ex.forward(q, k, v, causal=True, check=True)
+        with pytest.raises(ex.ExattnError) as e2:
+            ex.backward(q, k, v, o, lse, do, causal=True, check=True)
+    finally:
+        lib.attn_debug_inject_stall(0)
+        lib.attn_set_wait_timeout_ns(0)
+    assert e1.value.status == _lib.ATTN_ERR_TIMEOUT and e2.value.status == _lib.ATTN_ERR_TIMEOUT
+    assert ex.device_status() == 0

@@ -67,3 +67,33 @@ def test_noalloc_rejects_problems_beyond_its_scratch(cuda_device):
     assert lib.attn_bwd_noalloc(*args, 1, 1009, 128, 128, 0.1, 0, None) == _lib.ATTN_ERR_INVALID
     assert lib.attn_bwd_noalloc(*args, 1, 32, 16384, 128, 0.1, 1, None) == _lib.ATTN_ERR_INVALID
     assert lib.attn_bwd_noalloc(*args, 1, 1, 8, 96, 0.1, 0, None) == _lib.ATTN_ERR_INVALID
+
+
+def test_noalloc_follows_a_device_reset(cuda_device, tmp_path):
+    """After cudaDeviceReset the context, and with it the scratch array, is
+    created anew, possibly at another address; the next attn_bwd_noalloc call
+    must use the new one.  Run in a child process that holds a single CUDA
+    runtime (a build of the library linked against the shared libcudart, no
+    torch), so the reset re-creates the context the library's kernels use."""
+    import json
+    import os
+    import subprocess
+    import sys
+
+    from exact_attention_106_b200 import build as b
+
+    cudart = "/usr/local/cuda/lib64/libcudart.so.12"
+    if not os.path.exists(cudart):
+        pytest.fail(f"{cudart} missing: cannot build the shared-runtime variant")
+    so = str(tmp_path / "libexattn_cudart_shared.so")
+    proc = subprocess.run(b.build_command(so, cudart="shared"), capture_output=True, text=True)
+    assert proc.returncode == 0, proc.stderr[-2000:]
+    child = os.path.join(os.path.dirname(os.path.abspath(__file__)), "noalloc_reset_child.py")
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES=os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0])
+    run = subprocess.run([sys.executable, child, cudart, so], capture_output=True, text=True, timeout=300, env=env)
+    assert run.returncode == 0, run.stdout[-2000:] + run.stderr[-2000:]
+    res = json.loads(run.stdout.strip().splitlines()[-1])
+    for phase in ("before", "after"):
+        # dK and dV have a fixed summation order; dQ's reduce-adds do not
+        assert res[phase]["dk"] == 0.0 and res[phase]["dv"] == 0.0, res
+        assert res[phase]["dq"] <= 5e-2, res
