@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME]
+    python bench.py --sweep [--sweep-points NAME,...]
 
 A step is one forward and one backward pass (every stage of the path) over one
 batch of the long-context workload, B=1, H=32, N=16384, d=128, causal, bf16
@@ -290,7 +291,11 @@ def run_ours(args, rank, world, local_rank):
     dkdv_tf = w.bwd_flops() / (mean["bwd_dkdv"] * 1e-3) / 1e12
     dominant = "bwd_dkdv" if mean["bwd_dkdv"] >= mean["fwd"] else "fwd"
     dom_tf = dkdv_tf if dominant == "bwd_dkdv" else fwd_tf
-    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    # The timed region is a fraction of a second to a few seconds of
+    # back-to-back launches: the burst peak is the denominator; the
+    # sustained one (seconds under the power cap) is reported beside it.
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     value = job_throughput(world, flops_step, args.steps, max_ms)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -308,13 +313,15 @@ def run_ours(args, rank, world, local_rank):
                    "step": "forward + backward (all stages)", "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (Q, K, V, dO 128 MiB each per step)"},
         "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
-        "pct_of_peak": {"fwd_of_measured_sustained": fwd_tf / peak, "bwd_of_measured_sustained": bwd_tf / peak,
+        "pct_of_peak": {"fwd_of_burst": fwd_tf / peak, "bwd_of_burst": bwd_tf / peak,
+                        "fwd_of_sustained": fwd_tf / peak_sus, "bwd_of_sustained": bwd_tf / peak_sus,
                         "fwd_of_spec_2250": fwd_tf / spec_peak, "bwd_of_spec_2250": bwd_tf / spec_peak,
                         "peak_source": peak_src},
         "kernels": {k_: {"mean_ms": mean[k_]} for k_ in mean},
         "roofline": {"kernel": "attn_bwd_kernel<128>" if dominant == "bwd_dkdv" else "attn_fwd_kernel<128>",
                      "bound": "tensor", "achieved": dom_tf, "peak": peak, "unit": "TFLOP/s",
-                     "frac": dom_tf / peak, "peak_kind": f"bf16 sustained ({peak_src})",
+                     "frac": dom_tf / peak, "peak_kind": f"bf16 burst ({peak_src})",
+                     "frac_of_sustained": dom_tf / peak_sus,
                      "traffic": recorded_traffic() if dominant == "bwd_dkdv" else None},
         "cpu_baseline": cpu,
         "e2e": {"value": job_throughput(world, flops_step, e2e_steps, e2e_ms), "unit": "TFLOP/s",
@@ -325,6 +332,98 @@ def run_ours(args, rank, world, local_rank):
     result["kernels"]["fwd"]["tflops"] = fwd_tf
     result["kernels"]["bwd_dkdv"]["tflops"] = dkdv_tf
     return result
+
+
+# ------------------------------------------------------------------ sweep
+SPEC_PEAK_TFLOPS = 2250.0  # dense bf16, B200 spec
+SM_COUNT = 148
+FLOP_PER_SM_CYCLE = 8192   # bf16 MMA rate of one SM (128x128x16 per 64 cycles)
+
+
+def sweep_workloads():
+    from exact_attention_106_b200 import workloads as W
+    return W.sweep() + [W.SINGLE_HEAD_32K, W.SINGLE_HEAD_32K_CAUSAL]
+
+
+def time_point(w, dev, min_reps: int, min_seconds: float, flush):
+    """Median and minimum CUDA-event time of the forward and of each backward
+    stage on workload w, with the L2 flushed (256 MiB write) before each
+    forward + backward repetition; repetitions are raised until the timed launches of the point last
+    at least `min_seconds`, so the clock samples cover them."""
+    import exact_attention_106_b200 as ex
+    from exact_attention_106_b200 import workloads as W
+    B, H, N, d = w.shape
+    q, k, v, do = (x.to(dev) for x in W.make_inputs(w))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    ws = ex.alloc_workspace(B, H, N, d, dev)
+    stream = torch.cuda.current_stream(dev)
+    names = ["fwd", "bwd_preprocess", "bwd_dkdv", "bwd_dq_convert"]
+
+    def rep():
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(8)]
+        flush.zero_()
+        evs[0].record(stream)
+        ex.forward(q, k, v, causal=w.causal, scale=w.softmax_scale, out=o, lse=lse)
+        evs[1].record(stream)
+        gen = ex.bwd_stages(q, k, v, o, lse, do, dq, dk, dv, ws, causal=w.causal, scale=w.softmax_scale)
+        for i in range(3):
+            evs[2 + 2 * i].record(stream)
+            next(gen)
+            evs[3 + 2 * i].record(stream)
+        return evs
+
+    for _ in range(3):
+        rep()
+    torch.cuda.synchronize(dev)
+    t0 = time.perf_counter()
+    evs = [rep()]
+    torch.cuda.synchronize(dev)
+    est = max(time.perf_counter() - t0, 1e-4)
+    reps = max(min_reps, int(min_seconds / est) + 1)
+    with ClockSampler(dev.index or 0) as clk:
+        evs = [rep() for _ in range(reps)]
+        torch.cuda.synchronize(dev)
+    if ex.device_status(dev) != 0:
+        raise RuntimeError(f"device status not clean after {w.name}")
+    ms = {n: sorted(e[2 * i].elapsed_time(e[2 * i + 1]) for e in evs) for i, n in enumerate(names)}
+    return {n: {"median_ms": statistics.median(v), "min_ms": v[0]} for n, v in ms.items()}, reps, clk.summary()
+
+
+def run_sweep(args):
+    """One JSON line per point of the sweep (fixed 16384 tokens per batch,
+    N in 512..16384, d in {64, 128}, causal and not) and of the single-head
+    N = 32768 d = 128 problems: forward and backward TFLOP/s and their
+    fractions of the burst, spec and clock-scaled tensor peaks."""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    only = set(args.sweep_points.split(",")) if args.sweep_points else None
+    rows = []
+    for w in sweep_workloads():
+        if only and w.name not in only:
+            continue
+        t, reps, clk = time_point(w, dev, args.sweep_reps, args.sweep_seconds, flush)
+        fwd_ms = t["fwd"]["median_ms"]
+        bwd_ms = t["bwd_preprocess"]["median_ms"] + t["bwd_dkdv"]["median_ms"] + t["bwd_dq_convert"]["median_ms"]
+        fwd_tf = w.fwd_flops() / (fwd_ms * 1e-3) / 1e12
+        bwd_tf = w.bwd_flops() / (bwd_ms * 1e-3) / 1e12
+        mhz = clk["sm_mhz"] if clk else None
+        clock_peak = SM_COUNT * FLOP_PER_SM_CYCLE * mhz * 1e6 / 1e12 if mhz else None
+        row = {"point": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "reps": reps,
+               "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "stages_ms": t,
+               "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
+               "fwd_of_burst": fwd_tf / burst, "bwd_of_burst": bwd_tf / burst,
+               "fwd_of_spec_2250": fwd_tf / SPEC_PEAK_TFLOPS, "bwd_of_spec_2250": bwd_tf / SPEC_PEAK_TFLOPS,
+               "fwd_of_clock_peak": fwd_tf / clock_peak if clock_peak else None,
+               "bwd_of_clock_peak": bwd_tf / clock_peak if clock_peak else None,
+               "burst_peak": burst, "peak_source": peak_src, "clocks": clk}
+        rows.append(row)
+        print(json.dumps(row), flush=True)
+    return rows
 
 
 # ------------------------------------------------------------ reference arm
@@ -367,6 +466,11 @@ def main(argv=None):
     ap.add_argument("--cpu-heads", type=int, default=3, help="full heads timed for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=2048, help="oracle sample size per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time every sweep point and the single-head 32K problems (one JSON line each)")
+    ap.add_argument("--sweep-points", default="", help="comma-separated subset of sweep point names")
+    ap.add_argument("--sweep-reps", type=int, default=10, help="minimum timed repetitions per point")
+    ap.add_argument("--sweep-seconds", type=float, default=0.5, help="minimum timed seconds per point")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -377,6 +481,11 @@ def main(argv=None):
     if world != args.gpus:
         ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
 
+    if args.sweep:
+        if world != 1 or args.impl != "ours":
+            ap.error("--sweep runs on one GPU, our implementation")
+        run_sweep(args)
+        return 0
     if args.impl == "reference":
         out = run_reference(args, rank)
     else:

@@ -8,8 +8,9 @@ used for device memory and streams.
     o, lse = forward(q, k, v, causal=False, scale=None)
     dq, dk, dv = backward(q, k, v, o, lse, do, causal=False, scale=None)
 
-Tensors are CUDA bfloat16, contiguous [B, H, N, d] with d in {64, 128};
-lse is float32 [B, H, N].  ``scale`` defaults to 1/sqrt(d).
+Tensors are CUDA bfloat16 (or float16, through the _fp16 entry points),
+contiguous [B, H, N, d] with d in {64, 128}; lse is float32 [B, H, N].
+``scale`` defaults to 1/sqrt(d).
 """
 from __future__ import annotations
 
@@ -30,13 +31,17 @@ def _stream(device: torch.device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
 
+# element type -> (forward, backward) entry points of the C ABI
+_ENTRY = {torch.bfloat16: ("attn_fwd", "attn_bwd"), torch.float16: ("attn_fwd_fp16", "attn_bwd_fp16")}
+
+
 def _check_qkv(*ts: torch.Tensor) -> None:
-    shape = ts[0].shape
+    shape, dtype = ts[0].shape, ts[0].dtype
     for t in ts:
-        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous() and t.dim() == 4):
-            raise ValueError("expected contiguous CUDA bfloat16 tensors [B, H, N, d]")
-        if t.shape != shape or t.device != ts[0].device:
-            raise ValueError("q, k, v (and o, do) must share shape and device")
+        if not (t.is_cuda and t.dtype in _ENTRY and t.is_contiguous() and t.dim() == 4):
+            raise ValueError("expected contiguous CUDA bfloat16 or float16 tensors [B, H, N, d]")
+        if t.shape != shape or t.device != ts[0].device or t.dtype != dtype:
+            raise ValueError("q, k, v (and o, do) must share shape, dtype and device")
 
 
 def _scale(d: int, scale: Optional[float]) -> float:
@@ -64,12 +69,12 @@ def forward(q, k, v, causal: bool = False, scale: Optional[float] = None, out=No
     B, H, N, d = q.shape
     o = torch.empty_like(q) if out is None else out
     lse_t = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
-    lib = _lib.load()
-    _lib.check("attn_fwd", lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                                        lse_t.data_ptr(), B, H, N, d, _scale(d, scale), int(causal),
-                                        _stream(q.device)))
+    name = _ENTRY[q.dtype][0]
+    _lib.check(name, getattr(_lib.load(), name)(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                               lse_t.data_ptr(), B, H, N, d, _scale(d, scale), int(causal),
+                                               _stream(q.device)))
     if check:
-        _check_status("attn_fwd", q.device)
+        _check_status(name, q.device)
     return o, lse_t
 
 
@@ -99,13 +104,13 @@ def backward(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] =
     else:
         dq, dk, dv = out
     ws = alloc_workspace(B, H, N, d, q.device) if workspace is None else workspace
-    lib = _lib.load()
-    _lib.check("attn_bwd", lib.attn_bwd(
+    name = _ENTRY[q.dtype][1]
+    _lib.check(name, getattr(_lib.load(), name)(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
         dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, _scale(d, scale), int(causal),
         ws.data_ptr(), ws.numel(), _stream(q.device)))
     if check:
-        _check_status("attn_bwd", q.device)
+        _check_status(name, q.device)
     return dq, dk, dv
 
 
@@ -113,7 +118,10 @@ def bwd_stages(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool = False,
                scale: Optional[float] = None):
     """The backward as three separate C-ABI calls (what ``backward`` runs), each
     returning after its launch; yields between stages so a caller can record
-    CUDA events around each."""
+    CUDA events around each.  bf16 only (the stages have no fp16 entry
+    points)."""
+    if q.dtype != torch.bfloat16:
+        raise ValueError("bwd_stages takes bfloat16 tensors")
     B, H, N, d = q.shape
     sc = _scale(d, scale)
     st = _stream(q.device)

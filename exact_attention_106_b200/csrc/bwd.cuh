@@ -13,15 +13,16 @@
 //   keeps K_j, V_j in shared memory and dK_j, dV_j in tensor memory, and walks
 //   the query tiles i (i >= j under the causal mask).  Per query tile:
 //     S^T = K_j Q_i^T            (tcgen05, TMEM)
-//     P^T = exp2(S^T c - LSE_i)  (registers -> TMEM as bf16, over S^T)
+//     P^T = exp2(S^T c - LSE_i)  (registers -> TMEM as 16-bit, over S^T)
 //     dP^T = V_j dO_i^T          (tcgen05, TMEM)
 //     dV_j += P^T dO_i           (A operand read from TMEM)
-//     dS^T = P^T o (dP^T - D_i)  (registers -> shared memory as bf16)
+//     dS^T = P^T o (dP^T - D_i)  (registers -> shared memory as 16-bit)
 //     dK_j += dS^T Q_i ;  dQ_i-partial = dS K_j  (tcgen05)
 //   and adds the dQ partial into the fp32 accumulator: four drain warps read
 //   it from tensor memory (handing the columns back at once), stage it in
 //   shared memory and let the TMA engine add it into global memory.
-// Stage 3 (attn_bwd_dq_convert_kernel): dQ = bf16(scale * accumulator).
+// Stage 3 (attn_bwd_dq_convert_kernel): dQ = T(scale * accumulator), T the element type
+// (bf16 or fp16; inputs, gradients, P and dS all use it).
 #pragma once
 #include "ptx.cuh"
 
@@ -33,8 +34,8 @@ struct BwdParams {
   CUtensorMap tm_v;
   CUtensorMap tm_do;
   CUtensorMap tm_dq;  // fp32 2-D {d, B*H*Np}, box {32, 32}, 128-byte swizzle (dQ accumulator)
-  __nv_bfloat16* dk;
-  __nv_bfloat16* dv;
+  void* dk;  // [B*H, N, d] of the element type T
+  void* dv;
   float* dq_acc;       // [BH, Np, d]
   const float* dvec;   // [BH, Np]  D
   const float* lse2;   // [BH, Np]  LSE * log2(e), +inf on padded rows
@@ -75,7 +76,7 @@ struct BwdCfg {
   static constexpr uint32_t kOffV = kTile;
   static constexpr uint32_t kOffQ = 2 * kTile;   // 2 stages
   static constexpr uint32_t kOffDO = 4 * kTile;  // 2 stages
-  static constexpr uint32_t kOffDS = 6 * kTile;  // 128 x 128 bf16
+  static constexpr uint32_t kOffDS = 6 * kTile;  // 128 x 128 16-bit
   static constexpr uint32_t kOffVec = kOffDS + 32768;  // 2 stages x (LSE2[128], D[128]) fp32
   // dQ staging: at d = 128 the dO buffer of the step being drained (dead once
   // dV and dP have read it); at d = 64 a buffer of its own (32 KB).
@@ -93,9 +94,9 @@ struct BwdCfg {
 
 // X[128 x 128] = A[128 x D] B[128 x D]^T with both operands K-major D-wide
 // tiles at offsets a0, b0 from the shared-memory base (S^T and dP^T).
-template <int D>
+template <int D, typename T>
 __device__ __forceinline__ void bwd_issue_t(uint32_t d_tmem, SmemDesc dKm, uint32_t a0, uint32_t b0) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
+  constexpr uint32_t idesc = idesc_16_f32(Elem<T>::kMmaFmt, 128, 128, 0, 0);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -103,9 +104,11 @@ __device__ __forceinline__ void bwd_issue_t(uint32_t d_tmem, SmemDesc dKm, uint3
   }
 }
 
-template <int D>
+// T: the 16-bit element type of Q, K, V, dO and the gradients.
+template <int D, typename T>
 __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant__ BwdParams p) {
   using C = BwdCfg<D>;
+  using E = Elem<T>;
   constexpr int kProducerWarp = 12;
   constexpr int kMmaWarp = 13;   // also allocates TMEM
   constexpr int kMmaWarp2 = 14;
@@ -147,13 +150,13 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int N = p.N;
-  const int T = p.ntiles;
+  const int ntq = p.ntiles;  // query tiles
   // Key tile 0 first (under the causal mask it sees the most query tiles), a
   // few heads at a time.
   int j, bh;
   grouped_order(static_cast<int>(blockIdx.x), p.ntiles, p.BH, p.head_group, j, bh);
   const int i0 = p.causal ? j : 0;
-  const int n = T - i0;  // >= 1
+  const int n = ntq - i0;  // >= 1
 
   if (threadIdx.x == 0) {
     mbar_init(bar_kv, 1);
@@ -241,8 +244,8 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
     // A commit covers only its own thread's MMAs; every hand-off between
     // the two goes through a barrier below.
     if (lane == 0) {
-      constexpr uint32_t idesc_kv = idesc_bf16_f32(128, D, 0, 1);  // dV, dK: B = dO / Q MN-major
-      constexpr uint32_t idesc_q = idesc_bf16_f32(128, D, 1, 1);   // dQ: A = dS MN-major, B = K MN-major
+      constexpr uint32_t idesc_kv = idesc_16_f32(E::kMmaFmt, 128, D, 0, 1);  // dV, dK: B = dO / Q MN-major
+      constexpr uint32_t idesc_q = idesc_16_f32(E::kMmaFmt, 128, D, 1, 1);   // dQ: A = dS MN-major, B = K MN-major
       // K-major and MN-major views of this CTA's shared memory, built once;
       // every operand below is an offset from the dynamic shared-memory base.
       const SmemDesc dKm = make_desc_sw128(smem_u32(smem), 16, 1024);
@@ -254,9 +257,9 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
                   mbar_wait(&bar_dofull[0], 0, abort_flag, tmo, 212);
         if (ok) {
           tc_fence_after();
-          bwd_issue_t<D>(tmem + C::kColS, dKm, oK, oQ);
+          bwd_issue_t<D, T>(tmem + C::kColS, dKm, oK, oQ);
           tc_commit(bar_s);
-          bwd_issue_t<D>(tmem + C::kColDP, dKm, oV, oDO);
+          bwd_issue_t<D, T>(tmem + C::kColDP, dKm, oV, oDO);
           tc_commit(bar_dp);
         }
         for (int it = 0; it < n && ok; ++it) {
@@ -276,7 +279,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
             // next S^T as early as possible: its softmax overlaps dQ, dK of tile it
             if (!mbar_wait(&bar_qfull[st1], ph1, abort_flag, tmo, 214)) break;
             tc_fence_after();
-            bwd_issue_t<D>(tmem + C::kColS, dKm, oK, oQ + st1 * TILE);
+            bwd_issue_t<D, T>(tmem + C::kColS, dKm, oK, oQ + st1 * TILE);
             tc_commit(bar_s);
             // dP^T(it+1) overwrites dP^T(it), read once dS_i is written, and at
             // d = 128 also the dQ partial, free once the drain has read it
@@ -284,7 +287,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
             if (D == 128 && !mbar_wait(bar_dqfree, it & 1, abort_flag, tmo, 217)) break;
             if (!mbar_wait(&bar_dofull[st1], ph1, abort_flag, tmo, 218)) break;
             tc_fence_after();
-            bwd_issue_t<D>(tmem + C::kColDP, dKm, oV, oDO + st1 * TILE);
+            bwd_issue_t<D, T>(tmem + C::kColDP, dKm, oV, oDO + st1 * TILE);
             tc_commit(bar_dp);
           }
         }
@@ -404,7 +407,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
           }
         }
       }
-      // bf16 P^T over the first 32 columns of this half's scores: query pair
+      // 16-bit P^T over the first 32 columns of this half's scores: query pair
       // 2m, 2m+1 of the half in column m (m = 4g + t%4)
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
@@ -413,7 +416,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
         for (int e = 0; e < 16; ++e) {
           float p0, p1;
           f2_unpack(pf[b][e], p0, p1);
-          pk[e] = pack_bf16x2(p0, p1);
+          pk[e] = E::pack2(p0, p1);
         }
         tmem_st16x128_x8(tS + (static_cast<uint32_t>(16 * b) << 16), pk);
       }
@@ -450,7 +453,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
                                                dd));
             float d0, d1;
             f2_unpack(ds2, d0, d1);
-            w[rr] = pack_bf16x2(d0, d1);
+            w[rr] = E::pack2(d0, d1);
           }
           // rows 32wq + 16b + (lane & 15): 8x8 matrices rr = 0, 1 of column group g
           stmatrix_x2(ds_lane + 16 * b * 128 + ((g ^ ds_sw) << 4), w[0], w[1]);
@@ -466,7 +469,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       const bool key_ok = key < N;
       const uint32_t tAcc = tmem + lane_off + (h == 0 ? C::kColDK : C::kColDV);
       const float mul = (h == 0) ? p.scale : 1.0f;
-      __nv_bfloat16* out = (h == 0 ? p.dk : p.dv) + (static_cast<size_t>(bh) * N + key) * D;
+      T* out = static_cast<T*>(h == 0 ? p.dk : p.dv) + (static_cast<size_t>(bh) * N + key) * D;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t a[32];
@@ -476,7 +479,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
           uint32_t w[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e)
-            w[e] = pack_bf16x2(__uint_as_float(a[2 * e]) * mul, __uint_as_float(a[2 * e + 1]) * mul);
+            w[e] = E::pack2(__uint_as_float(a[2 * e]) * mul, __uint_as_float(a[2 * e + 1]) * mul);
           uint4* dst = reinterpret_cast<uint4*>(out + 32 * cc);
 #pragma unroll
           for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
@@ -565,9 +568,8 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
 
 // ---------------------------------------------------------------- stage 1
 // One row per (d/8) lanes; each lane reads 8 elements (16 bytes) of O and dO.
-template <int D>
-__global__ void __launch_bounds__(256) attn_bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o,
-                                                                  const __nv_bfloat16* __restrict__ dO,
+template <int D, typename T>
+__global__ void __launch_bounds__(256) attn_bwd_preprocess_kernel(const T* __restrict__ o, const T* __restrict__ dO,
                                                                   const float* __restrict__ lse,
                                                                   float* __restrict__ dvec,
                                                                   float* __restrict__ lse2,
@@ -587,12 +589,11 @@ __global__ void __launch_bounds__(256) attn_bwd_preprocess_kernel(const __nv_bfl
     const size_t off = (static_cast<size_t>(bh) * N + i) * D + sub * 8;
     const uint4 a = *reinterpret_cast<const uint4*>(o + off);
     const uint4 b = *reinterpret_cast<const uint4*>(dO + off);
-    const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
-    const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
+    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float2 x = __bfloat1622float2(pa[e]);
-      const float2 y = __bfloat1622float2(pb[e]);
+      const float2 x = Elem<T>::unpack2(wa[e]);
+      const float2 y = Elem<T>::unpack2(wb[e]);
       acc = fmaf(x.x, y.x, acc);
       acc = fmaf(x.y, y.y, acc);
     }
@@ -610,23 +611,27 @@ __global__ void __launch_bounds__(256) attn_bwd_preprocess_kernel(const __nv_bfl
   }
 }
 
-inline void launch_bwd_preprocess(const __nv_bfloat16* o, const __nv_bfloat16* dO, const float* lse, float* dvec,
-                                  float* lse2, float* dq_acc, int BH, int N, int Np, int d, cudaStream_t s) {
+template <typename T>
+inline void launch_bwd_preprocess(const void* o, const void* dO, const float* lse, float* dvec, float* lse2,
+                                  float* dq_acc, int BH, int N, int Np, int d, cudaStream_t s) {
   const long long rows = static_cast<long long>(BH) * Np;
+  const T* ot = static_cast<const T*>(o);
+  const T* dt = static_cast<const T*>(dO);
   if (d == 64) {
     const unsigned blocks = static_cast<unsigned>((rows + 31) / 32);
-    attn_bwd_preprocess_kernel<64><<<blocks, 256, 0, s>>>(o, dO, lse, dvec, lse2, dq_acc, BH, N, Np);
+    attn_bwd_preprocess_kernel<64, T><<<blocks, 256, 0, s>>>(ot, dt, lse, dvec, lse2, dq_acc, BH, N, Np);
   } else {
     const unsigned blocks = static_cast<unsigned>((rows + 15) / 16);
-    attn_bwd_preprocess_kernel<128><<<blocks, 256, 0, s>>>(o, dO, lse, dvec, lse2, dq_acc, BH, N, Np);
+    attn_bwd_preprocess_kernel<128, T><<<blocks, 256, 0, s>>>(ot, dt, lse, dvec, lse2, dq_acc, BH, N, Np);
   }
 }
 
 // ---------------------------------------------------------------- stage 3
 // Each thread converts 8 consecutive elements of one row.
+template <typename T>
 __global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float* __restrict__ dq_acc,
-                                                                  __nv_bfloat16* __restrict__ dq, int N, int Np,
-                                                                  int d, float scale, long long total8) {
+                                                                  T* __restrict__ dq, int N, int Np, int d,
+                                                                  float scale, long long total8) {
   const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (t >= total8) return;
   const long long e = t * 8;                    // element index in [BH, N, d]
@@ -637,18 +642,19 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_convert_kernel(const float* _
   const float4* src = reinterpret_cast<const float4*>(dq_acc + (bh * Np + i) * d + col);
   const float4 a = src[0], b = src[1];
   uint4 w;
-  w.x = pack_bf16x2(a.x * scale, a.y * scale);
-  w.y = pack_bf16x2(a.z * scale, a.w * scale);
-  w.z = pack_bf16x2(b.x * scale, b.y * scale);
-  w.w = pack_bf16x2(b.z * scale, b.w * scale);
+  w.x = Elem<T>::pack2(a.x * scale, a.y * scale);
+  w.y = Elem<T>::pack2(a.z * scale, a.w * scale);
+  w.z = Elem<T>::pack2(b.x * scale, b.y * scale);
+  w.w = Elem<T>::pack2(b.z * scale, b.w * scale);
   *reinterpret_cast<uint4*>(dq + e) = w;
 }
 
-inline void launch_bwd_dq_convert(const float* dq_acc, __nv_bfloat16* dq, int BH, int N, int Np, int d, float scale,
+template <typename T>
+inline void launch_bwd_dq_convert(const float* dq_acc, void* dq, int BH, int N, int Np, int d, float scale,
                                   cudaStream_t s) {
   const long long total8 = static_cast<long long>(BH) * N * d / 8;
   const unsigned blocks = static_cast<unsigned>((total8 + 255) / 256);
-  attn_bwd_dq_convert_kernel<<<blocks, 256, 0, s>>>(dq_acc, dq, N, Np, d, scale, total8);
+  attn_bwd_dq_convert_kernel<T><<<blocks, 256, 0, s>>>(dq_acc, static_cast<T*>(dq), N, Np, d, scale, total8);
 }
 
 }  // namespace exattn

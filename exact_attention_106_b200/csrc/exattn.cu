@@ -8,6 +8,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "exattn.h"
 #include "ptx.cuh"
@@ -93,16 +94,22 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D view {d, N, B*H} of a contiguous bf16 [B,H,N,d] tensor; box {64, 128, 1}
-// with 128-byte swizzle.  Rows past N of a head read as zeros.
-bool make_map_bf16(CUtensorMap* m, const void* base, int BH, int N, int d) {
+template <typename T>
+constexpr CUtensorMapDataType map_type() {
+  return std::is_same<T, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+}
+
+// 3-D view {d, N, B*H} of a contiguous 16-bit [B,H,N,d] tensor; box
+// {64, 128, 1} with 128-byte swizzle.  Rows past N of a head read as zeros.
+template <typename T>
+bool make_map_16(CUtensorMap* m, const void* base, int BH, int N, int d) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
   cuuint32_t box[3] = {64, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+  return enc(m, map_type<T>(), 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -132,17 +139,16 @@ bool ensure_smem_attr(K kernel, int bytes) {
 // The backward kernel rebalances registers between warpgroups (setmaxnreg);
 // the split is only safe for a compiled register count in [kRegsMin, kRegsMax],
 // so a build outside that range is refused before its first launch.
-template <int D>
-bool bwd_regs_ok(int dev, std::atomic<int>* flags) {
-  if (flags[dev].load(std::memory_order_acquire)) return true;
+template <int D, typename T>
+bool bwd_regs_ok(int dev) {
+  static std::atomic<int> checked[kMaxDevices];  // one table per kernel instantiation
+  if (checked[dev].load(std::memory_order_acquire)) return true;
   cudaFuncAttributes a{};
-  if (cudaFuncGetAttributes(&a, exattn::attn_bwd_kernel<D>) != cudaSuccess) return false;
+  if (cudaFuncGetAttributes(&a, exattn::attn_bwd_kernel<D, T>) != cudaSuccess) return false;
   if (a.numRegs < exattn::BwdCfg<D>::kRegsMin || a.numRegs > exattn::BwdCfg<D>::kRegsMax) return false;
-  flags[dev].store(1, std::memory_order_release);
+  checked[dev].store(1, std::memory_order_release);
   return true;
 }
-std::atomic<int> g_bwd64_regs[kMaxDevices];
-std::atomic<int> g_bwd128_regs[kMaxDevices];
 
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH; }
@@ -156,11 +162,11 @@ int head_group(int BH, double per_head_bytes) {
   return g < 1.0 ? 1 : static_cast<int>(g);
 }
 
-}  // namespace
+// ------------------------------------------------------ typed implementations
+// T is the 16-bit element type of the tensors: __nv_bfloat16 or __half.
 
-extern "C" {
-
-int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+template <typename T>
+int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
              float scale, int causal, attn_stream_t stream) {
   const int sz = check_sizes(B, H, N, d);
   if (sz < 0 || !check_scale(scale)) return ATTN_ERR_INVALID;
@@ -174,10 +180,10 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   FwdParams p;
   std::memset(&p, 0, sizeof(p));
   const int BH = B * H;
-  if (!make_map_bf16(&p.tm_q, q, BH, N, d) || !make_map_bf16(&p.tm_k, k, BH, N, d) ||
-      !make_map_bf16(&p.tm_v, v, BH, N, d))
+  if (!make_map_16<T>(&p.tm_q, q, BH, N, d) || !make_map_16<T>(&p.tm_k, k, BH, N, d) ||
+      !make_map_16<T>(&p.tm_v, v, BH, N, d))
     return ATTN_ERR_LAUNCH;
-  p.o = static_cast<__nv_bfloat16*>(o);
+  p.o = o;
   p.lse = lse;
   p.N = N;
   p.BH = BH;
@@ -192,22 +198,18 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 64) {
     constexpr int smem = exattn::FwdCfg<64>::kSmem;
-    if (!ensure_smem_attr(exattn::attn_fwd_kernel<64>, smem)) return ATTN_ERR_LAUNCH;
-    exattn::attn_fwd_kernel<64><<<grid, exattn::FwdCfg<64>::kThreads, smem, s>>>(p);
+    if (!ensure_smem_attr(exattn::attn_fwd_kernel<64, T>, smem)) return ATTN_ERR_LAUNCH;
+    exattn::attn_fwd_kernel<64, T><<<grid, exattn::FwdCfg<64>::kThreads, smem, s>>>(p);
   } else {
     constexpr int smem = exattn::FwdCfg<128>::kSmem;
-    if (!ensure_smem_attr(exattn::attn_fwd_kernel<128>, smem)) return ATTN_ERR_LAUNCH;
-    exattn::attn_fwd_kernel<128><<<grid, exattn::FwdCfg<128>::kThreads, smem, s>>>(p);
+    if (!ensure_smem_attr(exattn::attn_fwd_kernel<128, T>, smem)) return ATTN_ERR_LAUNCH;
+    exattn::attn_fwd_kernel<128, T><<<grid, exattn::FwdCfg<128>::kThreads, smem, s>>>(p);
   }
   return launch_status();
 }
 
-size_t attn_bwd_workspace_bytes(int B, int H, int N, int d) {
-  if (check_sizes(B, H, N, d) != 0) return 0;
-  return workspace_bytes(B, H, N, d);
-}
-
-int attn_bwd_preprocess(const void* o, const void* dO, const float* lse, int B, int H, int N, int d,
+template <typename T>
+int preprocess_impl(const void* o, const void* dO, const float* lse, int B, int H, int N, int d,
                         void* workspace, size_t workspace_bytes_given, attn_stream_t stream) {
   const int sz = check_sizes(B, H, N, d);
   if (sz < 0) return ATTN_ERR_INVALID;
@@ -222,12 +224,12 @@ int attn_bwd_preprocess(const void* o, const void* dO, const float* lse, int B, 
   const int BH = B * H;
   const int np = static_cast<int>(padded_rows(N));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  exattn::launch_bwd_preprocess(static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse,
-                                ws.dvec, ws.lse2, ws.dq_acc, BH, N, np, d, s);
+  exattn::launch_bwd_preprocess<T>(o, dO, lse, ws.dvec, ws.lse2, ws.dq_acc, BH, N, np, d, s);
   return launch_status();
 }
 
-int attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, int B, int H,
+template <typename T>
+int dkdv_impl(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, int B, int H,
                   int N, int d, float scale, int causal, void* workspace, size_t workspace_bytes_given,
                   attn_stream_t stream) {
   const int sz = check_sizes(B, H, N, d);
@@ -244,12 +246,12 @@ int attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, v
   BwdParams p;
   std::memset(&p, 0, sizeof(p));
   const int BH = B * H;
-  if (!make_map_bf16(&p.tm_q, q, BH, N, d) || !make_map_bf16(&p.tm_k, k, BH, N, d) ||
-      !make_map_bf16(&p.tm_v, v, BH, N, d) || !make_map_bf16(&p.tm_do, dO, BH, N, d) ||
+  if (!make_map_16<T>(&p.tm_q, q, BH, N, d) || !make_map_16<T>(&p.tm_k, k, BH, N, d) ||
+      !make_map_16<T>(&p.tm_v, v, BH, N, d) || !make_map_16<T>(&p.tm_do, dO, BH, N, d) ||
       !make_map_f32_dq(&p.tm_dq, ws.dq_acc, static_cast<size_t>(BH) * padded_rows(N), d))
     return ATTN_ERR_LAUNCH;
-  p.dk = static_cast<__nv_bfloat16*>(dk);
-  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.dk = dk;
+  p.dv = dv;
   p.dq_acc = ws.dq_acc;
   p.dvec = ws.dvec;
   p.lse2 = ws.lse2;
@@ -267,19 +269,20 @@ int attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, v
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 64) {
     constexpr int smem = exattn::BwdCfg<64>::kSmem;
-    if (!bwd_regs_ok<64>(dev, g_bwd64_regs)) return ATTN_ERR_LAUNCH;
-    if (!ensure_smem_attr(exattn::attn_bwd_kernel<64>, smem)) return ATTN_ERR_LAUNCH;
-    exattn::attn_bwd_kernel<64><<<grid, exattn::BwdCfg<64>::kThreads, smem, s>>>(p);
+    if (!(bwd_regs_ok<64, T>(dev))) return ATTN_ERR_LAUNCH;
+    if (!ensure_smem_attr(exattn::attn_bwd_kernel<64, T>, smem)) return ATTN_ERR_LAUNCH;
+    exattn::attn_bwd_kernel<64, T><<<grid, exattn::BwdCfg<64>::kThreads, smem, s>>>(p);
   } else {
     constexpr int smem = exattn::BwdCfg<128>::kSmem;
-    if (!bwd_regs_ok<128>(dev, g_bwd128_regs)) return ATTN_ERR_LAUNCH;
-    if (!ensure_smem_attr(exattn::attn_bwd_kernel<128>, smem)) return ATTN_ERR_LAUNCH;
-    exattn::attn_bwd_kernel<128><<<grid, exattn::BwdCfg<128>::kThreads, smem, s>>>(p);
+    if (!(bwd_regs_ok<128, T>(dev))) return ATTN_ERR_LAUNCH;
+    if (!ensure_smem_attr(exattn::attn_bwd_kernel<128, T>, smem)) return ATTN_ERR_LAUNCH;
+    exattn::attn_bwd_kernel<128, T><<<grid, exattn::BwdCfg<128>::kThreads, smem, s>>>(p);
   }
   return launch_status();
 }
 
-int attn_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, const void* workspace,
+template <typename T>
+int dq_convert_impl(void* dq, int B, int H, int N, int d, float scale, const void* workspace,
                         size_t workspace_bytes_given, attn_stream_t stream) {
   const int sz = check_sizes(B, H, N, d);
   if (sz < 0 || !check_scale(scale)) return ATTN_ERR_INVALID;
@@ -291,23 +294,75 @@ int attn_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, const
   if (int st = check_device(&dev)) return st;
   const Workspace ws = carve(const_cast<void*>(workspace), B, H, N, d);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  exattn::launch_bwd_dq_convert(ws.dq_acc, static_cast<__nv_bfloat16*>(dq), B * H, N,
-                                static_cast<int>(padded_rows(N)), d, scale, s);
+  exattn::launch_bwd_dq_convert<T>(ws.dq_acc, dq, B * H, N, static_cast<int>(padded_rows(N)), d, scale, s);
   return launch_status();
 }
 
-int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+template <typename T>
+int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
              void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, void* workspace,
              size_t workspace_bytes_given, attn_stream_t stream) {
   const int sz = check_sizes(B, H, N, d);
   if (sz < 0 || !check_scale(scale)) return ATTN_ERR_INVALID;
   if (sz == 1) return ATTN_OK;
   if (!dq) return ATTN_ERR_INVALID;
-  int st = attn_bwd_preprocess(o, dO, lse, B, H, N, d, workspace, workspace_bytes_given, stream);
+  int st = preprocess_impl<T>(o, dO, lse, B, H, N, d, workspace, workspace_bytes_given, stream);
   if (st) return st;
-  st = attn_bwd_dkdv(q, k, v, dO, dk, dv, B, H, N, d, scale, causal, workspace, workspace_bytes_given, stream);
+  st = dkdv_impl<T>(q, k, v, dO, dk, dv, B, H, N, d, scale, causal, workspace, workspace_bytes_given, stream);
   if (st) return st;
-  return attn_bwd_dq_convert(dq, B, H, N, d, scale, workspace, workspace_bytes_given, stream);
+  return dq_convert_impl<T>(dq, B, H, N, d, scale, workspace, workspace_bytes_given, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+// ------------------------------------------------------------- bf16 entry points
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+             float scale, int causal, attn_stream_t stream) {
+  return fwd_impl<__nv_bfloat16>(q, k, v, o, lse, B, H, N, d, scale, causal, stream);
+}
+
+size_t attn_bwd_workspace_bytes(int B, int H, int N, int d) {
+  if (check_sizes(B, H, N, d) != 0) return 0;
+  return workspace_bytes(B, H, N, d);
+}
+
+int attn_bwd_preprocess(const void* o, const void* dO, const float* lse, int B, int H, int N, int d,
+                        void* workspace, size_t workspace_bytes_given, attn_stream_t stream) {
+  return preprocess_impl<__nv_bfloat16>(o, dO, lse, B, H, N, d, workspace, workspace_bytes_given, stream);
+}
+
+int attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, int B, int H,
+                  int N, int d, float scale, int causal, void* workspace, size_t workspace_bytes_given,
+                  attn_stream_t stream) {
+  return dkdv_impl<__nv_bfloat16>(q, k, v, dO, dk, dv, B, H, N, d, scale, causal, workspace,
+                                  workspace_bytes_given, stream);
+}
+
+int attn_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, const void* workspace,
+                        size_t workspace_bytes_given, attn_stream_t stream) {
+  return dq_convert_impl<__nv_bfloat16>(dq, B, H, N, d, scale, workspace, workspace_bytes_given, stream);
+}
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+             void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal, void* workspace,
+             size_t workspace_bytes_given, attn_stream_t stream) {
+  return bwd_impl<__nv_bfloat16>(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, workspace,
+                                 workspace_bytes_given, stream);
+}
+
+// ------------------------------------------------------------- fp16 entry points
+int attn_fwd_fp16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                  float scale, int causal, attn_stream_t stream) {
+  return fwd_impl<__half>(q, k, v, o, lse, B, H, N, d, scale, causal, stream);
+}
+
+int attn_bwd_fp16(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                  void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
+                  void* workspace, size_t workspace_bytes_given, attn_stream_t stream) {
+  return bwd_impl<__half>(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, workspace,
+                          workspace_bytes_given, stream);
 }
 
 void attn_set_wait_timeout_ns(unsigned long long ns) {

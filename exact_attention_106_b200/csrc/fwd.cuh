@@ -6,13 +6,15 @@
 //
 // One CTA owns a 256-row block of queries of one (batch, head), split into two
 // 128-row sub-tiles that ping-pong on the tensor core (while the softmax of
-// one sub-tile runs, the MMAs of the other do).  Roles (320 threads):
-//   warps 0..3    softmax of sub-tile 0 (one thread per query row)
-//   warps 4..7    softmax of sub-tile 1
-//   warp 8        TMA producer: Q (once), then K_j and V_j into a smem ring
-//   warp 9        TMEM allocator; lane 0 issues every tcgen05.mma
+// one sub-tile runs, the MMAs of the other do).  Roles (W = FwdCfg::kSoftmaxWG
+// softmax warpgroups, 128 W + 64 threads):
+//   warps 0..4W-1  softmax, one thread per query row: with W = 2 warps 0..3
+//                  serve sub-tile 0 and warps 4..7 sub-tile 1; with W = 1
+//                  warps 0..3 serve both, alternating step by step
+//   warp 4W        TMA producer: Q (once), then K_j and V_j into a smem ring
+//   warp 4W+1      TMEM allocator; lane 0 issues every tcgen05.mma
 // Tensor memory (512 columns x 128 lanes of 32 bit), per sub-tile k:
-//   columns [256k, 256k+128)      S_k = Q_k K_j^T (fp32); P_k (bf16 pairs) is
+//   columns [256k, 256k+128)      S_k = Q_k K_j^T (fp32); P_k (16-bit pairs) is
 //                                 written back over its first 64 columns
 //   columns [256k+128, +d)        O_k accumulator (fp32)
 // The softmax keeps, per row, a reference maximum and the running sum l;
@@ -30,7 +32,7 @@ struct FwdParams {
   CUtensorMap tm_q;  // 3-D {d, N, B*H}, box {64, 128, 1}, 128-byte swizzle
   CUtensorMap tm_k;
   CUtensorMap tm_v;
-  __nv_bfloat16* o;
+  void* o;  // [B*H, N, d] of the element type T
   float* lse;
   int N;
   int BH;
@@ -48,9 +50,30 @@ struct FwdParams {
 // d = 128 (one exp per score against 4*d flops of MMA).
 constexpr int kEmuPairs = 3;
 
+// Softmax warpgroups per CTA.  With 2, warpgroup k owns sub-tile k and the
+// two softmaxes run side by side; with 1, one warpgroup alternates between
+// the sub-tiles, so that each softmax has its SM sub-partitions to itself
+// while the other sub-tile's products run on the tensor core.
+#ifndef EXATTN_FWD_SOFTMAX_WG_D128
+#define EXATTN_FWD_SOFTMAX_WG_D128 2
+#endif
+#ifndef EXATTN_FWD_SOFTMAX_WG_D64
+#define EXATTN_FWD_SOFTMAX_WG_D64 2
+#endif
+
+#ifndef EXATTN_FWD_WAIT_KIND
+#define EXATTN_FWD_WAIT_KIND 0
+#endif
+#ifndef EXATTN_FWD_P_INTERLEAVE
+#define EXATTN_FWD_P_INTERLEAVE 0
+#endif
+constexpr int kFwdWaitKind = EXATTN_FWD_WAIT_KIND;
+
 template <int D>
 struct FwdCfg {
-  static constexpr int kThreads = 320;
+  static constexpr int kSoftmaxWG = (D == 128) ? EXATTN_FWD_SOFTMAX_WG_D128 : EXATTN_FWD_SOFTMAX_WG_D64;
+  static_assert(kSoftmaxWG == 1 || kSoftmaxWG == 2, "one or two softmax warpgroups");
+  static constexpr int kThreads = 128 * kSoftmaxWG + 64;
   static constexpr uint32_t kTile = 128u * D * 2u;  // one 128-row bf16 tile
   static constexpr int kSlots = (D == 128) ? 4 : 8;  // K/V ring slots
   static constexpr int kChunks = D / 64;             // 64-column swizzle chunks per tile
@@ -58,11 +81,13 @@ struct FwdCfg {
   static constexpr uint32_t kSmem = kBarOff + 256;
 };
 
-template <int D>
-__global__ void __launch_bounds__(320, 1) attn_fwd_kernel(const __grid_constant__ FwdParams p) {
+// T: the 16-bit element type of Q, K, V and O (__nv_bfloat16 or __half).
+template <int D, typename T>
+__global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1) attn_fwd_kernel(const __grid_constant__ FwdParams p) {
   using C = FwdCfg<D>;
-  constexpr int kProducerWarp = 8;
-  constexpr int kMmaWarp = 9;
+  using E = Elem<T>;
+  constexpr int kProducerWarp = 4 * C::kSoftmaxWG;
+  constexpr int kMmaWarp = kProducerWarp + 1;
   constexpr int SLOTS = C::kSlots;
   constexpr uint32_t TILE = C::kTile;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -87,7 +112,7 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_kernel(const __grid_constant_
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int N = p.N;
-  const int T = (N + 127) >> 7;
+  const int ntk = (N + 127) >> 7;  // key tiles
   // Heaviest query blocks first (they see the most keys under the causal
   // mask), a few heads at a time.
   int rank, bh;
@@ -97,7 +122,7 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_kernel(const __grid_constant_
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
     const int row0 = qb * 256 + k * 128;
-    n_sub[k] = (row0 >= N) ? 0 : (p.causal ? min(T, 2 * qb + k + 1) : T);
+    n_sub[k] = (row0 >= N) ? 0 : (p.causal ? min(ntk, 2 * qb + k + 1) : ntk);
   }
   const int nmax = max(n_sub[0], n_sub[1]);
 
@@ -177,8 +202,8 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_kernel(const __grid_constant_
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && nmax > 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);  // Q, K both K-major
-      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);    // P from TMEM, V MN-major
+      constexpr uint32_t idesc_s = idesc_16_f32(E::kMmaFmt, 128, 128, 0, 0);  // Q, K both K-major
+      constexpr uint32_t idesc_o = idesc_16_f32(E::kMmaFmt, 128, D, 0, 1);    // P from TMEM, V MN-major
       const uint32_t sq0 = smem_u32(sQ);
       const uint32_t skv0 = smem_u32(sKV);
       auto kslot = [&](int j) { return (2 * j) % SLOTS; };
@@ -207,8 +232,8 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_kernel(const __grid_constant_
           mma_ts(dt, at + kk * 8, desc_at(dMN, b0 + kk * 2048), idesc_o, (acc || kk > 0) ? 1u : 0u);
       };
       const int n0 = n_sub[0], n1 = n_sub[1];
-      bool ok = mbar_wait(bar_q, 0, abort_flag, tmo, 110);
-      ok = ok && mbar_wait(&bar_full[kslot(0)], kph(0), abort_flag, tmo, 111);
+      bool ok = mbar_wait_fast<kFwdWaitKind>(bar_q, 0, abort_flag, tmo, 110);
+      ok = ok && mbar_wait_fast<kFwdWaitKind>(&bar_full[kslot(0)], kph(0), abort_flag, tmo, 111);
       if (ok) {
         tc_fence_after();
         if (n0 > 0) {
@@ -223,16 +248,16 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_kernel(const __grid_constant_
       }
       for (int j = 0; j < nmax && ok; ++j) {
         const bool knext = (j + 1 < nmax);
-        if (!mbar_wait(&bar_full[vslot(j)], vph(j), abort_flag, tmo, 112)) break;
+        if (!mbar_wait_fast<kFwdWaitKind>(&bar_full[vslot(j)], vph(j), abort_flag, tmo, 112)) break;
         tc_fence_after();
         if (j < n0) {
-          if (!mbar_wait(&bar_p[0], j & 1, abort_flag, tmo, 113)) break;
+          if (!mbar_wait_fast<kFwdWaitKind>(&bar_p[0], j & 1, abort_flag, tmo, 113)) break;
           tc_fence_after();
           issue_pv(0, vslot(j), j > 0);
           if (j == n0 - 1) tc_commit(&bar_o[0]);
         }
         if (knext) {
-          if (!mbar_wait(&bar_full[kslot(j + 1)], kph(j + 1), abort_flag, tmo, 114)) break;
+          if (!mbar_wait_fast<kFwdWaitKind>(&bar_full[kslot(j + 1)], kph(j + 1), abort_flag, tmo, 114)) break;
           tc_fence_after();
         }
         if (j + 1 < n0) {
@@ -240,7 +265,7 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_kernel(const __grid_constant_
           tc_commit(&bar_s[0]);
         }
         if (j < n1) {
-          if (!mbar_wait(&bar_p[1], j & 1, abort_flag, tmo, 115)) break;
+          if (!mbar_wait_fast<kFwdWaitKind>(&bar_p[1], j & 1, abort_flag, tmo, 115)) break;
           tc_fence_after();
           issue_pv(1, vslot(j), j > 0);
           if (j == n1 - 1) tc_commit(&bar_o[1]);
@@ -259,24 +284,21 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_kernel(const __grid_constant_
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax
-    const int k = warp >> 2;        // sub-tile
-    const int wq = warp & 3;        // TMEM lane quadrant
+    const int wq = warp & 3;  // TMEM lane quadrant
     const int row = wq * 32 + lane;
-    const int q_row = qb * 256 + k * 128 + row;
-    const uint32_t tS = tmem + (static_cast<uint32_t>(wq * 32) << 16) + k * 256;
-    const uint32_t tO = tS + 128;
-    const int n = k ? n_sub[1] : n_sub[0];
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const float c = p.scale_log2;
     const float thr = 8.0f / c;  // reference max moves only if exps would exceed 2^8
-    float m_ref = -INFINITY;
-    float l = 0.f;
-    bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      // warp-uniform outcome: the tcgen05.ld/st below are warp-collective
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar_s[k], j & 1, abort_flag, tmo, 120 + k))) {
-        ok = false;
-        break;
-      }
+
+    // One step of the online softmax for sub-tile k, key tile j: load S_k,
+    // mask, move the reference maximum if needed (rescaling O_k), write P_k
+    // as bf16 over S_k and signal the MMA issuer.  Returns false if a wait
+    // gave up (the outcome is warp-uniform: the tcgen05.ld/st are
+    // warp-collective).
+    auto step = [&](int k, int j, float& m_ref, float& l) -> bool {
+      const uint32_t tS = lane_base + k * 256;
+      const uint32_t tO = tS + 128;
+      if (!__all_sync(0xffffffffu, mbar_wait_fast<kFwdWaitKind>(&bar_s[k], j & 1, abort_flag, tmo, 120 + k))) return false;
       tc_fence_after();
       uint32_t sr[128];
       tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
@@ -321,14 +343,18 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_kernel(const __grid_constant_
         suma[i & 1] = f2_add(suma[i & 1], pp);
         float p0, p1;
         f2_unpack(pp, p0, p1);
-        pk[i] = pack_bf16x2(p0, p1);
+        pk[i] = E::pack2(p0, p1);
+        if (EXATTN_FWD_P_INTERLEAVE && (i & 15) == 15)  // 32 probabilities ready: store them now
+          tmem_st16(tS + (i >> 4) * 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[i - 15]));
       }
       float s0, s1, s2, s3;
       f2_unpack(suma[0], s0, s1);
       f2_unpack(suma[1], s2, s3);
       l = l * alpha + ((s0 + s1) + (s2 + s3));
+      if (!EXATTN_FWD_P_INTERLEAVE) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) tmem_st16(tS + 16 * i, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * i]));
+        for (int i = 0; i < 4; ++i) tmem_st16(tS + 16 * i, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * i]));
+      }
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
@@ -344,11 +370,18 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_kernel(const __grid_constant_
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bar_p[k]);
-    }
-    if (ok && n > 0 && __all_sync(0xffffffffu, mbar_wait(&bar_o[k], 0, abort_flag, tmo, 122 + k))) {
+      return true;
+    };
+
+    // Epilogue of sub-tile k once its last P V product is done: O = O / l
+    // as bf16, LSE = m scale + ln l.
+    auto epilogue = [&](int k, float m_ref, float l) {
+      if (!__all_sync(0xffffffffu, mbar_wait_fast<kFwdWaitKind>(&bar_o[k], 0, abort_flag, tmo, 122 + k))) return;
       tc_fence_after();
+      const uint32_t tO = lane_base + k * 256 + 128;
+      const int q_row = qb * 256 + k * 128 + row;
       const float inv_l = 1.0f / l;
-      __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * N + q_row) * D;
+      T* orow = static_cast<T*>(p.o) + (static_cast<size_t>(bh) * N + q_row) * D;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
@@ -358,13 +391,34 @@ __global__ void __launch_bounds__(320, 1) attn_fwd_kernel(const __grid_constant_
           uint32_t w[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+            w[i] = E::pack2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
           uint4* dst = reinterpret_cast<uint4*>(orow + 32 * cc);
 #pragma unroll
           for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
         }
       }
       if (q_row < N) p.lse[static_cast<size_t>(bh) * N + q_row] = m_ref * p.scale + __logf(l);
+    };
+
+    if (C::kSoftmaxWG == 2) {
+      const int k = warp >> 2;
+      const int n = k ? n_sub[1] : n_sub[0];
+      float m_ref = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < n && ok; ++j) ok = step(k, j, m_ref, l);
+      if (ok && n > 0) epilogue(k, m_ref, l);
+    } else {
+      // one warpgroup, sub-tiles alternating: (0, j), (1, j), (0, j + 1), ...
+      float m_ref[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+      bool ok = true;
+      for (int j = 0; j < nmax && ok; ++j) {
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+          if (ok && j < n_sub[k]) ok = step(k, j, m_ref[k], l[k]);
+      }
+#pragma unroll
+      for (int k = 0; k < 2; ++k)
+        if (ok && n_sub[k] > 0) epilogue(k, m_ref[k], l[k]);
     }
   }
   tc_fence_before();

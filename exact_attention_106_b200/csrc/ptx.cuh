@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 namespace exattn {
 
@@ -92,6 +93,53 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       record_status(kDevStatusTimeout, site);
       *abort_flag = 1;
       return false;
+    }
+  }
+}
+
+// Variant of mbar_wait for the waits on a kernel's critical path: the
+// barrier is polled without the suspend-time hint (kind 1, a blocking poll of
+// the hardware's default length) or with non-blocking test_wait (kind 2), so
+// that the waiter resumes as soon as the phase completes.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar_addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar_addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_try_wait_nohint(uint32_t bar_addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar_addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+template <int KIND>
+__device__ __forceinline__ bool mbar_wait_fast(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                               uint64_t timeout_ns, unsigned int site) {
+  if (KIND == 0) return mbar_wait(bar, parity, abort_flag, timeout_ns, site);
+  const uint32_t a = smem_u32(bar);
+  auto poll = [&]() { return KIND == 1 ? mbar_try_wait_nohint(a, parity) : mbar_test_wait(a, parity); };
+  if (poll()) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t n = 0;; ++n) {
+    if (poll()) return true;
+    if ((n & 15u) == 15u) {  // the clock and the abort flag every 16 polls
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > timeout_ns) {
+        record_status(kDevStatusTimeout, site);
+        *abort_flag = 1;
+        return false;
+      }
     }
   }
 }
@@ -198,12 +246,13 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
-// Instruction descriptor, kind::f16 with bf16 A/B and fp32 accumulate.
-// a_mn / b_mn: 0 = K-major operand, 1 = MN-major operand.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn) {
+// Instruction descriptor, kind::f16 with 16-bit A/B (fp16: format 0, bf16:
+// format 1; both operands of one MMA have the same type) and fp32
+// accumulate.  a_mn / b_mn: 0 = K-major operand, 1 = MN-major operand.
+__host__ __device__ constexpr uint32_t idesc_16_f32(uint32_t ab_fmt, int M, int N, int a_mn, int b_mn) {
   return (1u << 4)                          // D format: f32
-         | (1u << 7)                        // A format: bf16
-         | (1u << 10)                       // B format: bf16
+         | (ab_fmt << 7)                    // A format
+         | (ab_fmt << 10)                   // B format
          | (uint32_t(a_mn) << 15)           // A major
          | (uint32_t(b_mn) << 16)           // B major
          | (uint32_t(N >> 3) << 17)         // N / 8
@@ -431,5 +480,32 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // .x (low 16 bits) = lo
   return *reinterpret_cast<uint32_t*>(&h);
 }
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);  // .x (low 16 bits) = lo
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// The 16-bit input/output element types: bf16 (the default) and fp16.  The
+// kernels are written once; this gives the tensor-core operand format, the
+// round-to-nearest-even packing of two fp32 values, and the widening of a
+// packed pair.
+template <typename T>
+struct Elem;
+template <>
+struct Elem<__nv_bfloat16> {
+  static constexpr uint32_t kMmaFmt = 1;
+  __device__ static __forceinline__ uint32_t pack2(float lo, float hi) { return pack_bf16x2(lo, hi); }
+  __device__ static __forceinline__ float2 unpack2(uint32_t w) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
+  }
+};
+template <>
+struct Elem<__half> {
+  static constexpr uint32_t kMmaFmt = 0;
+  __device__ static __forceinline__ uint32_t pack2(float lo, float hi) { return pack_f16x2(lo, hi); }
+  __device__ static __forceinline__ float2 unpack2(uint32_t w) {
+    return __half22float2(*reinterpret_cast<const __half2*>(&w));
+  }
+};
 
 }  // namespace exattn

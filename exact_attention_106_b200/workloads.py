@@ -67,16 +67,18 @@ def _seeded_normal(shape, seed: int) -> torch.Tensor:
     return torch.randn(shape, generator=g, dtype=torch.float32)
 
 
-def make_inputs(w: Workload, with_grad_out: bool = True):
-    """Return (q, k, v, do) as contiguous CPU bfloat16 tensors [B,H,N,d]."""
+def make_inputs(w: Workload, with_grad_out: bool = True, dtype: torch.dtype = torch.bfloat16):
+    """Return (q, k, v, do) as contiguous CPU tensors [B,H,N,d] of ``dtype``
+    (bfloat16 by default; float16 for the fp16 path), each rounded to
+    nearest-even from the same float32 draw."""
     q = _seeded_normal(w.shape, w.seed_base + 0)
     if w.q_boost_heads_from is not None:
         q[:, w.q_boost_heads_from:] *= w.q_boost
     k = _seeded_normal(w.shape, w.seed_base + 1)
     v = _seeded_normal(w.shape, w.seed_base + 2)
-    out = [q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)]
+    out = [q.to(dtype), k.to(dtype), v.to(dtype)]
     if with_grad_out:
-        out.append(_seeded_normal(w.shape, w.seed_base + 3).to(torch.bfloat16))
+        out.append(_seeded_normal(w.shape, w.seed_base + 3).to(dtype))
     else:
         out.append(None)
     return tuple(out)

@@ -27,7 +27,7 @@
  * Conventions shared by every entry point
  * ----------------------------------------
  *  - Tensors q, k, v, o, dO, dq, dk, dv are bf16 (passed as raw 16-bit
- *    patterns), contiguous, row-major [B, H, N, d]: the (batch, heads,
+ *    patterns; the _fp16 entry points take fp16 instead), contiguous, row-major [B, H, N, d]: the (batch, heads,
  *    seq_len, head_dim) order of the pages' PyTorch examples.  lse is fp32
  *    [B, H, N].  All of them are DEVICE pointers on the current CUDA device.
  *  - d must be 64 or 128.  N >= 1 is arbitrary (no multiple-of-tile rule).
@@ -124,6 +124,25 @@ int attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, v
 /* Stage 3: dq = bf16(scale * dQ accumulator). */
 int attn_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, const void* workspace,
                         size_t workspace_bytes, attn_stream_t stream);
+
+/*
+ * fp16 inputs.  The same operations on IEEE half-precision tensors: q, k, v,
+ * o, dO, dq, dk, dv are fp16 (raw 16-bit patterns) instead of bf16; every
+ * other argument, the layout and the rules are those of attn_fwd and
+ * attn_bwd above (the same workspace size).  The probabilities P and the
+ * score gradients dS that feed the tensor cores are rounded to fp16, the
+ * accumulators stay fp32.  The pages list FP16 beside BF16 for every version
+ * of the method ("Walk through the FlashAttention algorithm ...", the
+ * v1/v2/v3 comparison table, precision row).  No range check is made: as
+ * with any fp16 computation, scores or gradients beyond the fp16 range
+ * (65504) overflow.
+ */
+int attn_fwd_fp16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                  float scale, int causal, attn_stream_t stream);
+
+int attn_bwd_fp16(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                  void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
+                  void* workspace, size_t workspace_bytes, attn_stream_t stream);
 
 /*
  * Backward without any device allocation: attn_bwd() run on scratch memory

@@ -42,15 +42,19 @@ def _const(path, name):
     return int(m.group(1))
 
 
-def _kernel(regs, stem, d, params):
-    name = f"_ZN6exattn{len(stem)}{stem}ILi{d}EEEvNS_{len(params)}{params}E"
+ELEMS = ["13__nv_bfloat16", "6__half"]  # mangled element types the kernels are instantiated for
+
+
+def _kernel(regs, stem, d, params, elem):
+    name = f"_ZN6exattn{len(stem)}{stem}ILi{d}E{elem}EEvNS_{len(params)}{params}E"
     assert name in regs, sorted(regs)
     return regs[name]
 
 
+@pytest.mark.parametrize("elem", ELEMS)
 @pytest.mark.parametrize("d", [64, 128])
-def test_backward_register_split_fits(registers, d):
-    r = _kernel(registers, "attn_bwd_kernel", d, "BwdParams")
+def test_backward_register_split_fits(registers, d, elem):
+    r = _kernel(registers, "attn_bwd_kernel", d, "BwdParams", elem)
     threads = _const("bwd.cuh", "kThreads")
     drain, side = _const("bwd.cuh", "kRegsDrain"), _const("bwd.cuh", "kRegsSide")
     # warpgroup 2 (drain) rises from r to `drain`, warpgroup 3 falls from r to `side`
@@ -61,8 +65,12 @@ def test_backward_register_split_fits(registers, d):
     assert 32 * (2 * r + drain + side) <= 16384
 
 
+@pytest.mark.parametrize("elem", ELEMS)
 @pytest.mark.parametrize("d", [64, 128])
-def test_forward_fits_the_sub_partitions(registers, d):
-    r = _kernel(registers, "attn_fwd_kernel", d, "FwdParams")
-    per_sub = math.ceil(_const("fwd.cuh", "kThreads") // 32 / 4)
+def test_forward_fits_the_sub_partitions(registers, d, elem):
+    r = _kernel(registers, "attn_fwd_kernel", d, "FwdParams", elem)
+    m = re.search(r"#define EXATTN_FWD_SOFTMAX_WG_D%d (\d+)" % d, open(os.path.join(CSRC, "fwd.cuh")).read())
+    assert m
+    threads = 128 * int(m.group(1)) + 64  # softmax warpgroups + producer and MMA warps
+    per_sub = math.ceil(threads // 32 / 4)
     assert per_sub * 32 * r <= 16384, (r, per_sub)
