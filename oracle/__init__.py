@@ -3,4 +3,4 @@
 TEST INFRASTRUCTURE ONLY: used by the test suite, ``__graft_entry__.smoke()``
 and the CPU-baseline leg of ``bench.py``.  The product path never imports it.
 """
-from .attention import backward, backward_head, forward, forward_head  # noqa: F401
+from .attention import backward, backward_head, decode, decode_head, forward, forward_head  # noqa: F401

@@ -143,3 +143,36 @@ def backward(q, k, v, do, scale: float, causal: bool, heads=None):
         for key, val in r.items():
             out[key][b, h] = val
     return out
+
+
+# ---------------------------------------------------------------------------
+# Decode: a few new queries against a long key/value history.
+#
+# The serving use the pages name ("Walk through the FlashAttention algorithm
+# ...", the paragraph on products: vLLM / TensorRT-LLM; "11.11 Flash
+# Attention", §Using Flash Attention, "vLLM") runs attention for the last Nq
+# positions of a sequence of Nk tokens.  It is the same definition with a
+# rectangular score matrix; under the causal mask the Nq queries are the LAST
+# Nq positions, so query i (0-based among the Nq) sees key j iff
+# j <= Nk - Nq + i (bottom-right alignment; for Nq = Nk it is the square mask
+# used above).  The pages do not state the alignment; this is the reading.
+# ---------------------------------------------------------------------------
+def decode_head(q, k, v, scale: float, causal: bool):
+    """One (batch, head): q [Nq,d], k,v [Nk,d] -> (O [Nq,d], LSE [Nq]) in float64."""
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    nq, nk = q.shape[0], k.shape[0]
+    # the queries sit at absolute positions nk - nq .. nk - 1
+    p, lse = _softmax_rows(_scores(q, k, scale, nk - nq, causal))
+    return p @ v, lse
+
+
+def decode(q, k, v, scale: float, causal: bool, heads=None):
+    """Whole tensors q [B,H,Nq,d], k/v [B,H,Nk,d], or only the listed (b, h)
+    pairs; returns (O [B,H,Nq,d], LSE [B,H,Nq]) as float64, NaN elsewhere."""
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    B, H, nq, d = q.shape
+    o = np.full((B, H, nq, d), np.nan)
+    lse = np.full((B, H, nq), np.nan)
+    for b, h in (heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]):
+        o[b, h], lse[b, h] = decode_head(q[b, h], k[b, h], v[b, h], scale, causal)
+    return o, lse
