@@ -6,13 +6,11 @@
 //
 // One CTA owns a 256-row block of queries of one (batch, head), split into two
 // 128-row sub-tiles that ping-pong on the tensor core (while the softmax of
-// one sub-tile runs, the MMAs of the other do).  Roles (W = FwdCfg::kSoftmaxWG
-// softmax warpgroups, 128 W + 64 threads):
-//   warps 0..4W-1  softmax, one thread per query row: with W = 2 warps 0..3
-//                  serve sub-tile 0 and warps 4..7 sub-tile 1; with W = 1
-//                  warps 0..3 serve both, alternating step by step
-//   warp 4W        TMA producer: Q (once), then K_j and V_j into a smem ring
-//   warp 4W+1      TMEM allocator; lane 0 issues every tcgen05.mma
+// one sub-tile runs, the MMAs of the other do).  Roles (320 threads):
+//   warps 0..3    softmax of sub-tile 0 (one thread per query row)
+//   warps 4..7    softmax of sub-tile 1
+//   warp 8        TMA producer: Q (once), then K_j and V_j into a smem ring
+//   warp 9        TMEM allocator; lane 0 issues every tcgen05.mma
 // Tensor memory (512 columns x 128 lanes of 32 bit), per sub-tile k:
 //   columns [256k, 256k+128)      S_k = Q_k K_j^T (fp32); P_k (16-bit pairs) is
 //                                 written back over its first 64 columns
@@ -50,30 +48,9 @@ struct FwdParams {
 // d = 128 (one exp per score against 4*d flops of MMA).
 constexpr int kEmuPairs = 3;
 
-// Softmax warpgroups per CTA.  With 2, warpgroup k owns sub-tile k and the
-// two softmaxes run side by side; with 1, one warpgroup alternates between
-// the sub-tiles, so that each softmax has its SM sub-partitions to itself
-// while the other sub-tile's products run on the tensor core.
-#ifndef EXATTN_FWD_SOFTMAX_WG_D128
-#define EXATTN_FWD_SOFTMAX_WG_D128 2
-#endif
-#ifndef EXATTN_FWD_SOFTMAX_WG_D64
-#define EXATTN_FWD_SOFTMAX_WG_D64 2
-#endif
-
-#ifndef EXATTN_FWD_WAIT_KIND
-#define EXATTN_FWD_WAIT_KIND 0
-#endif
-#ifndef EXATTN_FWD_P_INTERLEAVE
-#define EXATTN_FWD_P_INTERLEAVE 0
-#endif
-constexpr int kFwdWaitKind = EXATTN_FWD_WAIT_KIND;
-
 template <int D>
 struct FwdCfg {
-  static constexpr int kSoftmaxWG = (D == 128) ? EXATTN_FWD_SOFTMAX_WG_D128 : EXATTN_FWD_SOFTMAX_WG_D64;
-  static_assert(kSoftmaxWG == 1 || kSoftmaxWG == 2, "one or two softmax warpgroups");
-  static constexpr int kThreads = 128 * kSoftmaxWG + 64;
+  static constexpr int kThreads = 320;  // 8 softmax warps, producer warp, MMA warp
   static constexpr uint32_t kTile = 128u * D * 2u;  // one 128-row bf16 tile
   static constexpr int kSlots = (D == 128) ? 4 : 8;  // K/V ring slots
   static constexpr int kChunks = D / 64;             // 64-column swizzle chunks per tile
@@ -86,8 +63,8 @@ template <int D, typename T>
 __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1) attn_fwd_kernel(const __grid_constant__ FwdParams p) {
   using C = FwdCfg<D>;
   using E = Elem<T>;
-  constexpr int kProducerWarp = 4 * C::kSoftmaxWG;
-  constexpr int kMmaWarp = kProducerWarp + 1;
+  constexpr int kProducerWarp = 8;
+  constexpr int kMmaWarp = 9;
   constexpr int SLOTS = C::kSlots;
   constexpr uint32_t TILE = C::kTile;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -232,8 +209,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1) attn_fwd_kernel(const 
           mma_ts(dt, at + kk * 8, desc_at(dMN, b0 + kk * 2048), idesc_o, (acc || kk > 0) ? 1u : 0u);
       };
       const int n0 = n_sub[0], n1 = n_sub[1];
-      bool ok = mbar_wait_fast<kFwdWaitKind>(bar_q, 0, abort_flag, tmo, 110);
-      ok = ok && mbar_wait_fast<kFwdWaitKind>(&bar_full[kslot(0)], kph(0), abort_flag, tmo, 111);
+      bool ok = mbar_wait(bar_q, 0, abort_flag, tmo, 110);
+      ok = ok && mbar_wait(&bar_full[kslot(0)], kph(0), abort_flag, tmo, 111);
       if (ok) {
         tc_fence_after();
         if (n0 > 0) {
@@ -248,24 +225,24 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1) attn_fwd_kernel(const 
       }
       for (int j = 0; j < nmax && ok; ++j) {
         const bool knext = (j + 1 < nmax);
-        if (!mbar_wait_fast<kFwdWaitKind>(&bar_full[vslot(j)], vph(j), abort_flag, tmo, 112)) break;
+        // V_j and K_(j+1) have long landed by now; their waits come before the
+        // wait for P_0(j), so that no barrier wait sits between P_0 V_j and
+        // S_0(j+1) on sub-tile 0's critical path
+        if (!mbar_wait(&bar_full[vslot(j)], vph(j), abort_flag, tmo, 112)) break;
+        if (knext && !mbar_wait(&bar_full[kslot(j + 1)], kph(j + 1), abort_flag, tmo, 114)) break;
         tc_fence_after();
         if (j < n0) {
-          if (!mbar_wait_fast<kFwdWaitKind>(&bar_p[0], j & 1, abort_flag, tmo, 113)) break;
+          if (!mbar_wait(&bar_p[0], j & 1, abort_flag, tmo, 113)) break;
           tc_fence_after();
           issue_pv(0, vslot(j), j > 0);
           if (j == n0 - 1) tc_commit(&bar_o[0]);
-        }
-        if (knext) {
-          if (!mbar_wait_fast<kFwdWaitKind>(&bar_full[kslot(j + 1)], kph(j + 1), abort_flag, tmo, 114)) break;
-          tc_fence_after();
         }
         if (j + 1 < n0) {
           issue_s(0, kslot(j + 1));
           tc_commit(&bar_s[0]);
         }
         if (j < n1) {
-          if (!mbar_wait_fast<kFwdWaitKind>(&bar_p[1], j & 1, abort_flag, tmo, 115)) break;
+          if (!mbar_wait(&bar_p[1], j & 1, abort_flag, tmo, 115)) break;
           tc_fence_after();
           issue_pv(1, vslot(j), j > 0);
           if (j == n1 - 1) tc_commit(&bar_o[1]);
@@ -298,7 +275,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1) attn_fwd_kernel(const 
     auto step = [&](int k, int j, float& m_ref, float& l) -> bool {
       const uint32_t tS = lane_base + k * 256;
       const uint32_t tO = tS + 128;
-      if (!__all_sync(0xffffffffu, mbar_wait_fast<kFwdWaitKind>(&bar_s[k], j & 1, abort_flag, tmo, 120 + k))) return false;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar_s[k], j & 1, abort_flag, tmo, 120 + k))) return false;
       tc_fence_after();
       uint32_t sr[128];
       tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
@@ -344,17 +321,13 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1) attn_fwd_kernel(const 
         float p0, p1;
         f2_unpack(pp, p0, p1);
         pk[i] = E::pack2(p0, p1);
-        if (EXATTN_FWD_P_INTERLEAVE && (i & 15) == 15)  // 32 probabilities ready: store them now
-          tmem_st16(tS + (i >> 4) * 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[i - 15]));
       }
       float s0, s1, s2, s3;
       f2_unpack(suma[0], s0, s1);
       f2_unpack(suma[1], s2, s3);
       l = l * alpha + ((s0 + s1) + (s2 + s3));
-      if (!EXATTN_FWD_P_INTERLEAVE) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) tmem_st16(tS + 16 * i, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * i]));
-      }
+      for (int i = 0; i < 4; ++i) tmem_st16(tS + 16 * i, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * i]));
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
@@ -376,7 +349,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1) attn_fwd_kernel(const 
     // Epilogue of sub-tile k once its last P V product is done: O = O / l
     // as bf16, LSE = m scale + ln l.
     auto epilogue = [&](int k, float m_ref, float l) {
-      if (!__all_sync(0xffffffffu, mbar_wait_fast<kFwdWaitKind>(&bar_o[k], 0, abort_flag, tmo, 122 + k))) return;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar_o[k], 0, abort_flag, tmo, 122 + k))) return;
       tc_fence_after();
       const uint32_t tO = lane_base + k * 256 + 128;
       const int q_row = qb * 256 + k * 128 + row;
@@ -400,26 +373,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1) attn_fwd_kernel(const 
       if (q_row < N) p.lse[static_cast<size_t>(bh) * N + q_row] = m_ref * p.scale + __logf(l);
     };
 
-    if (C::kSoftmaxWG == 2) {
-      const int k = warp >> 2;
-      const int n = k ? n_sub[1] : n_sub[0];
-      float m_ref = -INFINITY, l = 0.f;
-      bool ok = true;
-      for (int j = 0; j < n && ok; ++j) ok = step(k, j, m_ref, l);
-      if (ok && n > 0) epilogue(k, m_ref, l);
-    } else {
-      // one warpgroup, sub-tiles alternating: (0, j), (1, j), (0, j + 1), ...
-      float m_ref[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
-      bool ok = true;
-      for (int j = 0; j < nmax && ok; ++j) {
-#pragma unroll
-        for (int k = 0; k < 2; ++k)
-          if (ok && j < n_sub[k]) ok = step(k, j, m_ref[k], l[k]);
-      }
-#pragma unroll
-      for (int k = 0; k < 2; ++k)
-        if (ok && n_sub[k] > 0) epilogue(k, m_ref[k], l[k]);
-    }
+    const int k = warp >> 2;  // sub-tile
+    const int n = k ? n_sub[1] : n_sub[0];
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n && ok; ++j) ok = step(k, j, m_ref, l);
+    if (ok && n > 0) epilogue(k, m_ref, l);
   }
   tc_fence_before();
   __syncthreads();

@@ -97,53 +97,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
-// Variant of mbar_wait for the waits on a kernel's critical path: the
-// barrier is polled without the suspend-time hint (kind 1, a blocking poll of
-// the hardware's default length) or with non-blocking test_wait (kind 2), so
-// that the waiter resumes as soon as the phase completes.
-__device__ __forceinline__ bool mbar_test_wait(uint32_t bar_addr, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(bar_addr), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ bool mbar_try_wait_nohint(uint32_t bar_addr, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(bar_addr), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-template <int KIND>
-__device__ __forceinline__ bool mbar_wait_fast(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                               uint64_t timeout_ns, unsigned int site) {
-  if (KIND == 0) return mbar_wait(bar, parity, abort_flag, timeout_ns, site);
-  const uint32_t a = smem_u32(bar);
-  auto poll = [&]() { return KIND == 1 ? mbar_try_wait_nohint(a, parity) : mbar_test_wait(a, parity); };
-  if (poll()) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t n = 0;; ++n) {
-    if (poll()) return true;
-    if ((n & 15u) == 15u) {  // the clock and the abort flag every 16 polls
-      if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > timeout_ns) {
-        record_status(kDevStatusTimeout, site);
-        *abort_flag = 1;
-        return false;
-      }
-    }
-  }
-}
-
 // Bounded wait (0.2 s) for the error path: lets copies or MMAs already in
 // flight finish before the CTA exits; ignores the abort flag.
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsigned int site) {

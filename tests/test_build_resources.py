@@ -69,8 +69,5 @@ def test_backward_register_split_fits(registers, d, elem):
 @pytest.mark.parametrize("d", [64, 128])
 def test_forward_fits_the_sub_partitions(registers, d, elem):
     r = _kernel(registers, "attn_fwd_kernel", d, "FwdParams", elem)
-    m = re.search(r"#define EXATTN_FWD_SOFTMAX_WG_D%d (\d+)" % d, open(os.path.join(CSRC, "fwd.cuh")).read())
-    assert m
-    threads = 128 * int(m.group(1)) + 64  # softmax warpgroups + producer and MMA warps
-    per_sub = math.ceil(threads // 32 / 4)
+    per_sub = math.ceil(_const("fwd.cuh", "kThreads") // 32 / 4)
     assert per_sub * 32 * r <= 16384, (r, per_sub)
