@@ -423,7 +423,84 @@ def run_sweep(args):
                "burst_peak": burst, "peak_source": peak_src, "clocks": clk}
         rows.append(row)
         print(json.dumps(row), flush=True)
+    for row in kvsplit_points(dev, flush, burst, peak_src, args, only):
+        rows.append(row)
+        print(json.dumps(row), flush=True)
     return rows
+
+
+def time_fn(fn, dev, flush, min_reps: int, min_seconds: float):
+    """Median / min CUDA-event time of fn() with the L2 flushed before each
+    call, and the clocks sampled while the timed calls run."""
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize(dev)
+    t0 = time.perf_counter()
+    fn()
+    torch.cuda.synchronize(dev)
+    reps = max(min_reps, int(min_seconds / max(time.perf_counter() - t0, 1e-4)) + 1)
+    evs = []
+    with ClockSampler(dev.index or 0) as clk:
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            flush.zero_()
+            a.record(stream)
+            fn()
+            b.record(stream)
+            evs.append((a, b))
+        torch.cuda.synchronize(dev)
+    ms = sorted(a.elapsed_time(b) for a, b in evs)
+    return statistics.median(ms), ms[0], reps, clk.summary()
+
+
+def kvsplit_points(dev, flush, burst, peak_src, args, only):
+    """The split-key forward (attn_fwd_kvsplit): the single-head 32K causal
+    problem, and the decode workloads (bandwidth-bound: GB/s of algorithmic
+    HBM bytes against the HBM peak)."""
+    import exact_attention_106_b200 as ex
+    from exact_attention_106_b200 import workloads as W
+    peaks, _ = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    out = []
+    w = W.SINGLE_HEAD_32K_CAUSAL
+    name = w.name + "_kvsplit"
+    if not only or name in only:
+        q, k, v, _ = (x.to(dev) if x is not None else None for x in W.make_inputs(w, with_grad_out=False))
+        splits, need = ex.kvsplit_plan(w.B, w.H, w.N, w.N, w.d, True, 0)
+        ws = torch.empty(max(1, need), dtype=torch.uint8, device=dev)
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+        med, mn, reps, clk = time_fn(lambda: ex.forward_kvsplit(q, k, v, causal=True, scale=w.softmax_scale,
+                                                               workspace=ws, out=o, lse=lse), dev, flush,
+                                     args.sweep_reps, args.sweep_seconds)
+        tf = w.fwd_flops() / (med * 1e-3) / 1e12
+        mhz = clk["sm_mhz"] if clk else None
+        out.append({"point": name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": True, "splits": splits,
+                    "reps": reps, "fwd_ms": med, "fwd_min_ms": mn, "fwd_tflops": tf, "fwd_of_burst": tf / burst,
+                    "fwd_of_spec_2250": tf / SPEC_PEAK_TFLOPS,
+                    "fwd_of_clock_peak": tf / (SM_COUNT * FLOP_PER_SM_CYCLE * mhz * 1e-6) if mhz else None,
+                    "burst_peak": burst, "peak_source": peak_src, "clocks": clk})
+    for w in W.DECODES:
+        if only and w.name not in only:
+            continue
+        q, k, v = (x.to(dev) for x in W.make_decode_inputs(w))
+        splits, need = ex.kvsplit_plan(w.B, w.H, w.Nq, w.Nk, w.d, w.causal, 0)
+        ws = torch.empty(max(1, need), dtype=torch.uint8, device=dev)
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+        med, mn, reps, clk = time_fn(lambda: ex.forward_kvsplit(q, k, v, causal=w.causal, scale=w.softmax_scale,
+                                                               workspace=ws, out=o, lse=lse), dev, flush,
+                                     args.sweep_reps, args.sweep_seconds)
+        gbs = w.bytes_moved() / (med * 1e-3) / 1e9
+        out.append({"point": w.name, "B": w.B, "H": w.H, "Nq": w.Nq, "Nk": w.Nk, "d": w.d, "causal": w.causal,
+                    "splits": splits, "reps": reps, "fwd_ms": med, "fwd_min_ms": mn,
+                    "fwd_tflops": w.fwd_flops() / (med * 1e-3) / 1e12, "bytes": w.bytes_moved(),
+                    "workspace_bytes": need, "gbs": gbs, "hbm_peak_gbs": hbm, "frac_of_hbm": gbs / hbm,
+                    "clocks": clk})
+        del q, k, v, ws, o, lse
+        torch.cuda.empty_cache()
+    return out
 
 
 # ------------------------------------------------------------ reference arm

@@ -21,7 +21,7 @@ import torch
 
 from . import _lib
 
-__all__ = ["forward", "backward", "forward_backward_host", "bwd_workspace_bytes", "host_buffer_bytes",
+__all__ = ["forward", "backward", "forward_kvsplit", "kvsplit_plan", "forward_backward_host", "bwd_workspace_bytes", "host_buffer_bytes",
            "device_status", "ExattnError"]
 
 ExattnError = _lib.ExattnError
@@ -75,6 +75,43 @@ def forward(q, k, v, causal: bool = False, scale: Optional[float] = None, out=No
                                                _stream(q.device)))
     if check:
         _check_status(name, q.device)
+    return o, lse_t
+
+
+def kvsplit_plan(B: int, H: int, Nq: int, Nk: int, d: int, causal: bool = False, splits: int = 0):
+    """(number of key ranges, workspace bytes) that ``forward_kvsplit`` uses."""
+    lib = _lib.load()
+    return (int(lib.attn_fwd_kvsplit_count(B, H, Nq, Nk, d, int(causal), splits)),
+            int(lib.attn_fwd_kvsplit_workspace_bytes(B, H, Nq, Nk, d, int(causal), splits)))
+
+
+def forward_kvsplit(q, k, v, causal: bool = False, scale: Optional[float] = None, splits: int = 0,
+                    workspace: Optional[torch.Tensor] = None, out=None, lse=None, check: bool = False):
+    """Forward over Nq queries and Nk keys with the keys split into ranges
+    (attn_fwd_kvsplit): decode (Nq small, Nk long) and long rows.
+
+    q: [B, H, Nq, d], k, v: [B, H, Nk, d], CUDA bfloat16, contiguous.  Under
+    ``causal`` the queries are the last Nq positions (query i sees keys
+    j <= Nk - Nq + i).  ``splits`` 0 lets the library choose.
+    """
+    for t in (q, k, v):
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous() and t.dim() == 4):
+            raise ValueError("expected contiguous CUDA bfloat16 tensors [B, H, N, d]")
+    B, H, Nq, d = q.shape
+    if k.shape != (B, H, k.shape[2], d) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, H, Nk, d] with q's B, H, d")
+    Nk = k.shape[2]
+    o = torch.empty_like(q) if out is None else out
+    lse_t = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device) if lse is None else lse
+    _, need = kvsplit_plan(B, H, Nq, Nk, d, causal, splits)
+    ws = workspace
+    if ws is None:
+        ws = torch.empty(max(1, need), dtype=torch.uint8, device=q.device)
+    _lib.check("attn_fwd_kvsplit", _lib.load().attn_fwd_kvsplit(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse_t.data_ptr(), B, H, Nq, Nk, d,
+        _scale(d, scale), int(causal), int(splits), ws.data_ptr(), ws.numel(), _stream(q.device)))
+    if check:
+        _check_status("attn_fwd_kvsplit", q.device)
     return o, lse_t
 
 

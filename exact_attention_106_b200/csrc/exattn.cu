@@ -9,6 +9,11 @@
 #include <cstring>
 #include <mutex>
 #include <type_traits>
+#include <algorithm>
+#include <map>
+#include <queue>
+#include <tuple>
+#include <vector>
 
 #include "exattn.h"
 #include "ptx.cuh"
@@ -165,6 +170,26 @@ int head_group(int BH, double per_head_bytes) {
 // ------------------------------------------------------ typed implementations
 // T is the 16-bit element type of the tensors: __nv_bfloat16 or __half.
 
+// Launches the forward kernel for a filled-in parameter block (tensor maps
+// and sizes set by the caller).
+template <typename T>
+int launch_fwd(FwdParams& p, int d, int dev, cudaStream_t s) {
+  p.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
+  p.debug_flags = g_debug_flags.load(std::memory_order_relaxed);
+  const dim3 grid(static_cast<unsigned>(p.nblocks) * static_cast<unsigned>(p.splits) * static_cast<unsigned>(p.BH));
+  (void)dev;
+  if (d == 64) {
+    constexpr int smem = exattn::FwdCfg<64>::kSmem;
+    if (!ensure_smem_attr(exattn::attn_fwd_kernel<64, T>, smem)) return ATTN_ERR_LAUNCH;
+    exattn::attn_fwd_kernel<64, T><<<grid, exattn::FwdCfg<64>::kThreads, smem, s>>>(p);
+  } else {
+    constexpr int smem = exattn::FwdCfg<128>::kSmem;
+    if (!ensure_smem_attr(exattn::attn_fwd_kernel<128, T>, smem)) return ATTN_ERR_LAUNCH;
+    exattn::attn_fwd_kernel<128, T><<<grid, exattn::FwdCfg<128>::kThreads, smem, s>>>(p);
+  }
+  return launch_status();
+}
+
 template <typename T>
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
              float scale, int causal, attn_stream_t stream) {
@@ -186,25 +211,171 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.o = o;
   p.lse = lse;
   p.N = N;
+  p.Nk = N;
+  p.q_off = 0;
   p.BH = BH;
   p.nblocks = (N + 255) / 256;
+  p.splits = 1;
+  p.tps = (N + 127) / 128;
   p.head_group = head_group(BH, 2.0 * N * d * 2);  // K and V of one head
   p.causal = causal ? 1 : 0;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
-  p.debug_flags = g_debug_flags.load(std::memory_order_relaxed);
-  const dim3 grid(static_cast<unsigned>(p.nblocks) * static_cast<unsigned>(BH));
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 64) {
-    constexpr int smem = exattn::FwdCfg<64>::kSmem;
-    if (!ensure_smem_attr(exattn::attn_fwd_kernel<64, T>, smem)) return ATTN_ERR_LAUNCH;
-    exattn::attn_fwd_kernel<64, T><<<grid, exattn::FwdCfg<64>::kThreads, smem, s>>>(p);
-  } else {
-    constexpr int smem = exattn::FwdCfg<128>::kSmem;
-    if (!ensure_smem_attr(exattn::attn_fwd_kernel<128, T>, smem)) return ATTN_ERR_LAUNCH;
-    exattn::attn_fwd_kernel<128, T><<<grid, exattn::FwdCfg<128>::kThreads, smem, s>>>(p);
+  return launch_fwd<T>(p, d, dev, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------ split-key forward
+constexpr int kMaxSplits = 64;
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+// Key tiles that query block qb (256 rows) sees: all of them, or under the
+// causal mask those up to the last visible key of its last row.
+int block_tiles(int qb, int Nq, int Nk, int causal) {
+  const int ntk = (Nk + 127) / 128;
+  const int last = std::min(qb * 256 + 255, Nq - 1);
+  return causal ? std::min(ntk, (last + (Nk - Nq)) / 128 + 1) : ntk;
+}
+
+// Number of key ranges per query block.  Enough CTAs for the machine come
+// from the (batch, head, query block) grid when it holds four or more waves:
+// then 1.  Otherwise each candidate S is simulated: the CTAs, in launch order
+// (heaviest query block first), are handed to the SMs as they free up, a CTA
+// costing its key tiles plus a fixed start-up cost, and S > 1 pays for the
+// merge pass; the S with the shortest makespan wins.  The result depends only
+// on the sizes and the SM count and is cached.
+int choose_splits(int BH, int Nq, int Nk, int causal) {
+  const int sms = sm_count();
+  const int nblocks = (Nq + 255) / 256;
+  const int ntk = (Nk + 127) / 128;
+  if (static_cast<long long>(BH) * nblocks >= 4LL * sms || ntk == 1) return 1;
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int, int, int>, int> cache;
+  const auto key = std::make_tuple(BH, Nq, Nk, causal, sms);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
   }
+  constexpr double kStartup = 2.5;  // per CTA, in units of one key tile's time
+  int best = 1;
+  double best_cost = 0;
+  for (int S = 1; S <= std::min(kMaxSplits, ntk); ++S) {
+    const int tps = (ntk + S - 1) / S;
+    const int se = (ntk + tps - 1) / tps;  // ranges actually distinct
+    if (se != S) continue;
+    if (static_cast<long long>(BH) * nblocks * S > 16LL * sms) break;
+    std::priority_queue<double, std::vector<double>, std::greater<double>> free_at;
+    for (int i = 0; i < sms; ++i) free_at.push(0.0);
+    double makespan = 0;
+    for (int r = 0; r < nblocks * S; ++r) {
+      const int qb = nblocks - 1 - r / S, sp = r % S;
+      const int cnt = std::max(0, std::min(block_tiles(qb, Nq, Nk, causal) - sp * tps, tps));
+      for (int h = 0; h < BH; ++h) {
+        const double t = free_at.top() + cnt + kStartup;
+        free_at.pop();
+        free_at.push(t);
+        makespan = std::max(makespan, t);
+      }
+    }
+    // the merge reads and writes (d + 1) fp32 per row and range: a few tiles' time
+    const double cost = makespan + (S > 1 ? 3.0 + 1e-6 * BH * static_cast<double>(Nq) * S : 0.0);
+    if (S == 1 || cost < best_cost) {
+      best = S;
+      best_cost = cost;
+    }
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  cache[key] = best;
+  return best;
+}
+
+// Resolves the split count (0 = automatic) and the key tiles per range.
+void resolve_splits(int BH, int Nq, int Nk, int causal, int requested, int* splits, int* tps) {
+  const int ntk = (Nk + 127) / 128;
+  int S = requested > 0 ? std::min(requested, kMaxSplits) : choose_splits(BH, Nq, Nk, causal);
+  S = std::max(1, std::min(S, ntk));
+  const int t = (ntk + S - 1) / S;
+  *tps = t;
+  *splits = (ntk + t - 1) / t;
+}
+
+size_t round_up256(size_t x) { return (x + 255) / 256 * 256; }
+
+size_t kvsplit_ws_bytes(int BH, int Nq, int d, int S) {
+  if (S <= 1) return 0;
+  const size_t rows = static_cast<size_t>(BH) * S * Nq;
+  return round_up256(rows * d * 4) + round_up256(rows * 4);
+}
+
+int check_kvsplit_sizes(int B, int H, int Nq, int Nk, int d, int causal, int splits) {
+  if (Nk < 0 || splits < 0) return -1;
+  const int sz = check_sizes(B, H, Nq, d);
+  if (sz != 0) return sz;
+  if (Nk == 0) return -1;             // a query with no keys has no softmax
+  if (causal && Nq > Nk) return -1;  // the first rows would see no key
+  const long long units = static_cast<long long>(B) * H * ((Nq + 255) / 256) * kMaxSplits;
+  if (units > 0x7fffffffLL) return -1;
+  return 0;
+}
+
+template <typename T>
+int kvsplit_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
+                 int d, float scale, int causal, int splits, void* workspace, size_t workspace_bytes_given,
+                 attn_stream_t stream) {
+  const int sz = check_kvsplit_sizes(B, H, Nq, Nk, d, causal, splits);
+  if (sz < 0 || !check_scale(scale)) return ATTN_ERR_INVALID;
+  if (sz == 1) return ATTN_OK;
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return ATTN_ERR_INVALID;
+  int dev = 0;
+  if (int st = check_device(&dev)) return st;
+  const int BH = B * H;
+  int S = 1, tps = 1;
+  resolve_splits(BH, Nq, Nk, causal ? 1 : 0, splits, &S, &tps);
+  const size_t need = kvsplit_ws_bytes(BH, Nq, d, S);
+  if (need > 0 && (!workspace || workspace_bytes_given < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)))
+    return ATTN_ERR_INVALID;
+
+  FwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  if (!make_map_16<T>(&p.tm_q, q, BH, Nq, d) || !make_map_16<T>(&p.tm_k, k, BH, Nk, d) ||
+      !make_map_16<T>(&p.tm_v, v, BH, Nk, d))
+    return ATTN_ERR_LAUNCH;
+  p.o = o;
+  p.lse = lse;
+  p.N = Nq;
+  p.Nk = Nk;
+  p.q_off = Nk - Nq;
+  p.BH = BH;
+  p.nblocks = (Nq + 255) / 256;
+  p.splits = S;
+  p.tps = tps;
+  if (S > 1) {
+    const size_t rows = static_cast<size_t>(BH) * S * Nq;
+    p.part_o = static_cast<float*>(workspace);
+    p.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + round_up256(rows * d * 4));
+  }
+  p.head_group = head_group(BH, 2.0 * Nk * d * 2);
+  p.causal = causal ? 1 : 0;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (int st = launch_fwd<T>(p, d, dev, s)) return st;
+  if (S == 1) return ATTN_OK;
+  const long long rows = static_cast<long long>(BH) * Nq;
+  const unsigned blocks = static_cast<unsigned>((rows + 7) / 8);
+  if (d == 64)
+    exattn::attn_fwd_merge_kernel<64, T><<<blocks, 256, 0, s>>>(p.part_o, p.part_lse, o, lse, BH, Nq, S);
+  else
+    exattn::attn_fwd_merge_kernel<128, T><<<blocks, 256, 0, s>>>(p.part_o, p.part_lse, o, lse, BH, Nq, S);
   return launch_status();
 }
 
@@ -350,6 +521,28 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
              size_t workspace_bytes_given, attn_stream_t stream) {
   return bwd_impl<__nv_bfloat16>(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, workspace,
                                  workspace_bytes_given, stream);
+}
+
+// ------------------------------------------------------------- split-key forward
+size_t attn_fwd_kvsplit_workspace_bytes(int B, int H, int Nq, int Nk, int d, int causal, int splits) {
+  if (check_kvsplit_sizes(B, H, Nq, Nk, d, causal, splits) != 0) return 0;
+  int S = 1, tps = 1;
+  resolve_splits(B * H, Nq, Nk, causal ? 1 : 0, splits, &S, &tps);
+  return kvsplit_ws_bytes(B * H, Nq, d, S);
+}
+
+int attn_fwd_kvsplit_count(int B, int H, int Nq, int Nk, int d, int causal, int splits) {
+  if (check_kvsplit_sizes(B, H, Nq, Nk, d, causal, splits) != 0) return 0;
+  int S = 1, tps = 1;
+  resolve_splits(B * H, Nq, Nk, causal ? 1 : 0, splits, &S, &tps);
+  return S;
+}
+
+int attn_fwd_kvsplit(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
+                     int Nk, int d, float scale, int causal, int splits, void* workspace,
+                     size_t workspace_bytes_given, attn_stream_t stream) {
+  return kvsplit_impl<__nv_bfloat16>(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, splits, workspace,
+                                     workspace_bytes_given, stream);
 }
 
 // ------------------------------------------------------------- fp16 entry points

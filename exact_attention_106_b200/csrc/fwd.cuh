@@ -28,13 +28,19 @@ namespace exattn {
 
 struct FwdParams {
   CUtensorMap tm_q;  // 3-D {d, N, B*H}, box {64, 128, 1}, 128-byte swizzle
-  CUtensorMap tm_k;
+  CUtensorMap tm_k;  // 3-D {d, Nk, B*H}, same boxes
   CUtensorMap tm_v;
   void* o;  // [B*H, N, d] of the element type T
   float* lse;
-  int N;
+  int N;      // query rows per head
+  int Nk;     // key rows per head (N for the square problem)
+  int q_off;  // Nk - N: the causal mask lets query row r see keys <= r + q_off
   int BH;
   int nblocks;  // ceil(N / 256)
+  int splits;   // key ranges per query block (1: the whole row, written as final output)
+  int tps;      // key tiles per range
+  float* part_o;    // splits > 1: [B*H, splits, N, d] fp32 partial O (normalised by its own l)
+  float* part_lse;  // splits > 1: [B*H, splits, N] fp32 partial LSE (-inf where the range saw no key)
   int head_group;  // heads whose CTAs are scheduled together (L2 reuse of K/V)
   int causal;
   float scale;       // softmax scale
@@ -89,17 +95,27 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1) attn_fwd_kernel(const 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int N = p.N;
-  const int ntk = (N + 127) >> 7;  // key tiles
+  const int Nk = p.Nk;
+  const int ntk = (Nk + 127) >> 7;  // key tiles
   // Heaviest query blocks first (they see the most keys under the causal
-  // mask), a few heads at a time.
+  // mask), a few heads at a time; the key ranges of one block side by side.
   int rank, bh;
-  grouped_order(static_cast<int>(blockIdx.x), p.nblocks, p.BH, p.head_group, rank, bh);
-  const int qb = p.nblocks - 1 - rank;
+  grouped_order(static_cast<int>(blockIdx.x), p.nblocks * p.splits, p.BH, p.head_group, rank, bh);
+  const int qb = p.nblocks - 1 - rank / p.splits;
+  const int split = rank % p.splits;
+  const int j0 = split * p.tps;  // first key tile of this CTA's range
+  // n_sub[k]: key tiles of this range that sub-tile k sees (all tiles up to
+  // the one holding the last visible key of its last row, within the range)
   int n_sub[2];
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
     const int row0 = qb * 256 + k * 128;
-    n_sub[k] = (row0 >= N) ? 0 : (p.causal ? min(ntk, 2 * qb + k + 1) : ntk);
+    int n = 0;
+    if (row0 < N) {
+      const int last = min(row0 + 127, N - 1);
+      n = p.causal ? min(ntk, (last + p.q_off) / 128 + 1) : ntk;
+    }
+    n_sub[k] = max(0, min(n - j0, p.tps));
   }
   const int nmax = max(n_sub[0], n_sub[1]);
 
@@ -159,7 +175,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1) attn_fwd_kernel(const 
           const CUtensorMap* m = x ? &p.tm_v : &p.tm_k;
 #pragma unroll
           for (int c = 0; c < C::kChunks; ++c)
-            tma_load_3d(sKV + slot * TILE + c * 16384, m, &bar_full[slot], c * 64, j * 128, bh);
+            tma_load_3d(sKV + slot * TILE + c * 16384, m, &bar_full[slot], c * 64, (j0 + j) * 128, bh);
 #pragma unroll
           for (int s = 0; s < SLOTS; ++s)
             if (s == slot) last_par[s] = static_cast<int>(ph);
@@ -283,10 +299,13 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1) attn_fwd_kernel(const 
       tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
       tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
       tmem_wait_ld();
-      const int key0 = j * 128;
-      const bool diag = p.causal && (j == 2 * qb + k);
-      if (diag || key0 + 128 > N) {
-        const int lim = min(diag ? row : 127, N - 1 - key0);  // last visible column
+      const int key0 = (j0 + j) * 128;
+      const int q_row = qb * 256 + k * 128 + row;
+      // masking is needed where the sub-tile's first row does not see the
+      // whole tile, or on the ragged last key tile
+      const bool part = p.causal && key0 + 127 > qb * 256 + k * 128 + p.q_off;
+      if (part || key0 + 128 > Nk) {
+        const int lim = min(part ? q_row + p.q_off - key0 : 127, Nk - 1 - key0);  // last visible column
 #pragma unroll
         for (int i = 0; i < 128; ++i)
           if (i > lim) sr[i] = __float_as_uint(-INFINITY);
@@ -353,6 +372,27 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1) attn_fwd_kernel(const 
       tc_fence_after();
       const uint32_t tO = lane_base + k * 256 + 128;
       const int q_row = qb * 256 + k * 128 + row;
+      if (p.part_o != nullptr) {
+        // one key range of a split row: O normalised by this range's own sum,
+        // and the range's logsumexp (-inf if the row saw none of its keys)
+        const float inv_l = l > 0.f ? 1.0f / l : 0.f;
+        const size_t prow = (static_cast<size_t>(bh) * p.splits + split) * N + q_row;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * cc, o);
+          tmem_wait_ld();
+          if (q_row < N) {
+            float4* dst = reinterpret_cast<float4*>(p.part_o + prow * D + 32 * cc);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv_l, __uint_as_float(o[4 * i + 1]) * inv_l,
+                                   __uint_as_float(o[4 * i + 2]) * inv_l, __uint_as_float(o[4 * i + 3]) * inv_l);
+          }
+        }
+        if (q_row < N) p.part_lse[prow] = l > 0.f ? m_ref * p.scale + __logf(l) : -INFINITY;
+        return;
+      }
       const float inv_l = 1.0f / l;
       T* orow = static_cast<T*>(p.o) + (static_cast<size_t>(bh) * N + q_row) * D;
 #pragma unroll
@@ -379,11 +419,78 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1) attn_fwd_kernel(const 
     bool ok = true;
     for (int j = 0; j < n && ok; ++j) ok = step(k, j, m_ref, l);
     if (ok && n > 0) epilogue(k, m_ref, l);
+    if (n == 0 && p.part_o != nullptr) {
+      // a range that holds none of this sub-tile's visible keys: an empty part
+      const int q_row = qb * 256 + k * 128 + row;
+      if (q_row < N) {
+        const size_t prow = (static_cast<size_t>(bh) * p.splits + split) * N + q_row;
+        float4* dst = reinterpret_cast<float4*>(p.part_o + prow * D);
+#pragma unroll
+        for (int i = 0; i < D / 4; ++i) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        p.part_lse[prow] = -INFINITY;
+      }
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace exattn
+
+namespace exattn {
+
+// Combines the key ranges of a split forward: per query row,
+//   LSE = log sum_s exp(LSE_s),  O = sum_s exp(LSE_s - LSE) O_s,
+// the merge of online-softmax partial results ("11.11 Flash Attention",
+// section "Flash Attention: The Key Insight": partial maxima and sums of
+// blocks combine exactly).  One warp per row; each lane holds d / 32 columns.
+template <int D, typename T>
+__global__ void __launch_bounds__(256) attn_fwd_merge_kernel(const float* __restrict__ part_o,
+                                                             const float* __restrict__ part_lse,
+                                                             void* __restrict__ o, float* __restrict__ lse, int BH,
+                                                             int N, int splits) {
+  constexpr int V = D / 32;  // columns per lane
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);  // over BH * N
+  const int lane = threadIdx.x & 31;
+  if (row >= static_cast<long long>(BH) * N) return;
+  const long long bh = row / N, i = row - bh * N;
+  float m = -INFINITY;
+  for (int s = 0; s < splits; ++s) m = fmaxf(m, part_lse[(bh * splits + s) * N + i]);
+  float acc[V];
+#pragma unroll
+  for (int c = 0; c < V; ++c) acc[c] = 0.f;
+  float wsum = 0.f;
+  if (m != -INFINITY) {
+    for (int s = 0; s < splits; ++s) {
+      const long long pr = (bh * splits + s) * N + i;
+      const float w = __expf(part_lse[pr] - m);
+      wsum += w;
+      const float* src = part_o + pr * D + lane * V;
+      if constexpr (V == 4) {
+        const float4 x = *reinterpret_cast<const float4*>(src);
+        acc[0] += w * x.x;
+        acc[1] += w * x.y;
+        acc[2] += w * x.z;
+        acc[3] += w * x.w;
+      } else {
+        const float2 x = *reinterpret_cast<const float2*>(src);
+        acc[0] += w * x.x;
+        acc[1] += w * x.y;
+      }
+    }
+  }
+  const float inv = wsum > 0.f ? 1.0f / wsum : 0.f;
+  uint32_t w2[V / 2];
+#pragma unroll
+  for (int c = 0; c < V / 2; ++c) w2[c] = Elem<T>::pack2(acc[2 * c] * inv, acc[2 * c + 1] * inv);
+  T* dst = static_cast<T*>(o) + row * D + lane * V;
+  if constexpr (V == 4)
+    *reinterpret_cast<uint2*>(dst) = make_uint2(w2[0], w2[1]);
+  else
+    *reinterpret_cast<uint32_t*>(dst) = w2[0];
+  if (lane == 0) lse[row] = (m == -INFINITY) ? -INFINITY : m + __logf(wsum);
 }
 
 }  // namespace exattn

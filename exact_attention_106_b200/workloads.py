@@ -118,8 +118,58 @@ SINGLE_HEAD_32K = Workload("single_head_1x1x32768x128_full", 1, 1, 32768, 128, F
 SINGLE_HEAD_32K_CAUSAL = Workload("single_head_1x1x32768x128_causal", 1, 1, 32768, 128, True, 6100)
 
 
-def by_name(name: str) -> Workload:
-    for w in NAMED + sweep() + [SINGLE_HEAD_32K, SINGLE_HEAD_32K_CAUSAL]:
+# ---------------------------------------------------------------------------
+# Decode: Nq new queries per head against Nk cached keys and values (the
+# serving use named on the pages: vLLM, TensorRT-LLM).  Q is [B, H, Nq, d],
+# K and V [B, H, Nk, d]; under the causal mask the queries are the last Nq
+# positions.  Same recipe: float32 N(0, 1) draws per tensor rounded to bf16.
+# ---------------------------------------------------------------------------
+@dataclasses.dataclass(frozen=True)
+class DecodeWorkload:
+    name: str
+    B: int
+    H: int
+    Nq: int
+    Nk: int
+    d: int
+    causal: bool
+    seed_base: int
+
+    @property
+    def softmax_scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def pairs(self) -> int:
+        if self.causal:  # query i sees Nk - Nq + i + 1 keys
+            per = self.Nq * (self.Nk - self.Nq) + self.Nq * (self.Nq + 1) // 2
+        else:
+            per = self.Nq * self.Nk
+        return self.B * self.H * per
+
+    def fwd_flops(self) -> int:
+        return 4 * self.d * self.pairs()
+
+    def bytes_moved(self) -> int:
+        """Algorithmic HBM bytes: read Q, K, V (bf16), write O (bf16) and LSE (fp32)."""
+        bh = self.B * self.H
+        return bh * (2 * self.Nq * self.d * 2 + 2 * self.Nk * self.d * 2 + self.Nq * 4)
+
+
+def make_decode_inputs(w: DecodeWorkload):
+    """(q, k, v) as contiguous CPU bfloat16 tensors."""
+    q = _seeded_normal((w.B, w.H, w.Nq, w.d), w.seed_base + 0)
+    k = _seeded_normal((w.B, w.H, w.Nk, w.d), w.seed_base + 1)
+    v = _seeded_normal((w.B, w.H, w.Nk, w.d), w.seed_base + 2)
+    return q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
+
+
+DECODE_1Q = DecodeWorkload("decode_8x32_q1_k32768x128_causal", 8, 32, 1, 32768, 128, True, 7000)
+DECODE_16Q = DecodeWorkload("decode_8x32_q16_k32768x128_causal", 8, 32, 16, 32768, 128, True, 7100)
+DECODES = [DECODE_1Q, DECODE_16Q]
+
+
+def by_name(name: str):
+    for w in NAMED + sweep() + [SINGLE_HEAD_32K, SINGLE_HEAD_32K_CAUSAL] + DECODES:
         if w.name == name:
             return w
     raise KeyError(name)

@@ -126,6 +126,45 @@ int attn_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, const
                         size_t workspace_bytes, attn_stream_t stream);
 
 /*
+ * Forward with the keys of each query row split into ranges: decode (a few
+ * new queries against a long key/value history) and long rows that leave the
+ * machine under-filled.
+ *
+ *   q, o  : bf16 [B,H,Nq,d] (in / out)     k, v : bf16 [B,H,Nk,d] (in)
+ *   lse   : fp32 [B,H,Nq] (out), natural-log logsumexp of each scaled score row
+ *   causal: the Nq queries are the LAST Nq positions of the Nk-token
+ *           sequence: query i sees key j iff j <= Nk - Nq + i (for Nq = Nk
+ *           the square mask of attn_fwd).  Requires Nq <= Nk.
+ *   splits: key ranges per query row; 0 lets the library choose (it simulates
+ *           the launch on the device's SM count), n > 0 asks for n (capped at
+ *           64 and at the number of 128-key tiles).
+ *   workspace: device, 256-byte aligned, >= attn_fwd_kvsplit_workspace_bytes()
+ *           with the same arguments (0 bytes, and NULL allowed, when a single
+ *           range is used); contents on entry are ignored.
+ *
+ * Each range is reduced tile by tile exactly as in attn_fwd, giving a partial
+ * output normalised by its own sum and its own logsumexp; a second kernel
+ * merges them, O = sum_s exp(LSE_s - LSE) O_s with LSE = log sum_s exp(LSE_s).
+ * This is the online-softmax algebra of "11.11 Flash Attention" (section
+ * "Flash Attention: The Key Insight") applied across ranges instead of
+ * tiles.  The serving use it exists for is named on the pages ("Walk through
+ * the FlashAttention algorithm ...", paragraph on products: vLLM, TensorRT-LLM).
+ * Nq = 0, B = 0 or H = 0 is an empty problem; Nk = 0 (no keys) is invalid.
+ * Same status codes as attn_fwd.
+ */
+int attn_fwd_kvsplit(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
+                     int Nk, int d, float scale, int causal, int splits, void* workspace, size_t workspace_bytes,
+                     attn_stream_t stream);
+
+/* Workspace bytes attn_fwd_kvsplit() needs for these arguments (0 if one
+ * range is used, or if the sizes are invalid or empty). */
+size_t attn_fwd_kvsplit_workspace_bytes(int B, int H, int Nq, int Nk, int d, int causal, int splits);
+
+/* The number of key ranges attn_fwd_kvsplit() uses for these arguments (0 if
+ * the sizes are invalid or empty). */
+int attn_fwd_kvsplit_count(int B, int H, int Nq, int Nk, int d, int causal, int splits);
+
+/*
  * fp16 inputs.  The same operations on IEEE half-precision tensors: q, k, v,
  * o, dO, dq, dk, dv are fp16 (raw 16-bit patterns) instead of bf16; every
  * other argument, the layout and the rules are those of attn_fwd and
