@@ -423,10 +423,43 @@ def run_sweep(args):
                "burst_peak": burst, "peak_source": peak_src, "clocks": clk}
         rows.append(row)
         print(json.dumps(row), flush=True)
-    for row in kvsplit_points(dev, flush, burst, peak_src, args, only):
+    for row in kvsplit_points(dev, flush, burst, peak_src, args, only) + fp8_points(dev, flush, burst, args, only):
         rows.append(row)
         print(json.dumps(row), flush=True)
     return rows
+
+
+def fp8_points(dev, flush, burst, args, only):
+    """The e4m3 forward (attn_fwd_fp8) on the d = 128 sweep shapes, causal and
+    not.  Its tensor-core peak is twice the bf16 one (the nominal ratio of
+    the dense e4m3 and bf16 rates, 4.5 / 2.25 PFLOP/s), applied to the
+    measured bf16 burst peak."""
+    import exact_attention_106_b200 as ex
+    from exact_attention_106_b200 import workloads as W
+    out = []
+    for w in [x for x in W.sweep() if x.d == 128 and x.N >= 4096] + [W.LONG_CONTEXT]:
+        name = w.name + "_fp8"
+        if only and name not in only:
+            continue
+        q, k, v, _ = W.make_inputs(w, with_grad_out=False, dtype=torch.float32)
+        sc = [float(t.abs().max()) / 448.0 for t in (q, k, v)]
+        q8, k8, v8 = ((t / s).to(torch.float8_e4m3fn).to(dev) for t, s in zip((q, k, v), sc))
+        del q, k, v
+        o = torch.empty(w.shape, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty(w.shape[:3], dtype=torch.float32, device=dev)
+        med, mn, reps, clk = time_fn(lambda: ex.forward_fp8(q8, k8, v8, *sc, causal=w.causal, scale=w.softmax_scale,
+                                                           out=o, lse=lse), dev, flush, args.sweep_reps,
+                                     args.sweep_seconds)
+        tf = w.fwd_flops() / (med * 1e-3) / 1e12
+        mhz = clk["sm_mhz"] if clk else None
+        out.append({"point": name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "reps": reps,
+                    "fwd_ms": med, "fwd_min_ms": mn, "fwd_tflops": tf, "fp8_peak": 2 * burst,
+                    "fwd_of_fp8_peak": tf / (2 * burst), "fwd_of_fp8_spec_4500": tf / 4500.0,
+                    "fwd_of_fp8_clock_peak": tf / (2 * SM_COUNT * FLOP_PER_SM_CYCLE * mhz * 1e-6) if mhz else None,
+                    "clocks": clk})
+        del q8, k8, v8, o, lse
+        torch.cuda.empty_cache()
+    return out
 
 
 def time_fn(fn, dev, flush, min_reps: int, min_seconds: float):

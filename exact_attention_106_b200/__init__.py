@@ -21,7 +21,7 @@ import torch
 
 from . import _lib
 
-__all__ = ["forward", "backward", "forward_kvsplit", "kvsplit_plan", "forward_backward_host", "bwd_workspace_bytes", "host_buffer_bytes",
+__all__ = ["forward", "backward", "forward_fp8", "forward_kvsplit", "kvsplit_plan", "forward_backward_host", "bwd_workspace_bytes", "host_buffer_bytes",
            "device_status", "ExattnError"]
 
 ExattnError = _lib.ExattnError
@@ -75,6 +75,27 @@ def forward(q, k, v, causal: bool = False, scale: Optional[float] = None, out=No
                                                _stream(q.device)))
     if check:
         _check_status(name, q.device)
+    return o, lse_t
+
+
+def forward_fp8(q, k, v, q_descale: float, k_descale: float, v_descale: float, causal: bool = False,
+                scale: Optional[float] = None, out=None, lse=None, check: bool = False):
+    """Forward on e4m3 inputs (attn_fwd_fp8): q, k, v CUDA float8_e4m3fn
+    [B, H, N, 128] whose real values are q * q_descale etc.  Returns
+    (o bf16, lse fp32)."""
+    for t in (q, k, v):
+        if not (t.is_cuda and t.dtype == torch.float8_e4m3fn and t.is_contiguous() and t.dim() == 4):
+            raise ValueError("expected contiguous CUDA float8_e4m3fn tensors [B, H, N, d]")
+        if t.shape != q.shape or t.device != q.device:
+            raise ValueError("q, k, v must share shape and device")
+    B, H, N, d = q.shape
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q.device) if out is None else out
+    lse_t = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    _lib.check("attn_fwd_fp8", _lib.load().attn_fwd_fp8(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse_t.data_ptr(), B, H, N, d, _scale(d, scale),
+        int(causal), float(q_descale), float(k_descale), float(v_descale), _stream(q.device)))
+    if check:
+        _check_status("attn_fwd_fp8", q.device)
     return o, lse_t
 
 

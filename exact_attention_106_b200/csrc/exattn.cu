@@ -101,18 +101,21 @@ EncodeTiledFn encode_fn() {
 
 template <typename T>
 constexpr CUtensorMapDataType map_type() {
+  if (sizeof(T) == 1) return CU_TENSOR_MAP_DATA_TYPE_UINT8;  // e4m3 bytes, copied as they are
   return std::is_same<T, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
 }
 
-// 3-D view {d, N, B*H} of a contiguous 16-bit [B,H,N,d] tensor; box
-// {64, 128, 1} with 128-byte swizzle.  Rows past N of a head read as zeros.
+// 3-D view {d, N, B*H} of a contiguous [B,H,N,d] tensor of T; box of 128
+// bytes by 128 rows by 1 with 128-byte swizzle.  Rows past N of a head read
+// as zeros.
 template <typename T>
 bool make_map_16(CUtensorMap* m, const void* base, int BH, int N, int d) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
+  constexpr cuuint64_t es = sizeof(T);
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * es, static_cast<cuuint64_t>(N) * d * es};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / es), 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, map_type<T>(), 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -178,14 +181,19 @@ int launch_fwd(FwdParams& p, int d, int dev, cudaStream_t s) {
   p.debug_flags = g_debug_flags.load(std::memory_order_relaxed);
   const dim3 grid(static_cast<unsigned>(p.nblocks) * static_cast<unsigned>(p.splits) * static_cast<unsigned>(p.BH));
   (void)dev;
-  if (d == 64) {
-    constexpr int smem = exattn::FwdCfg<64>::kSmem;
-    if (!ensure_smem_attr(exattn::attn_fwd_kernel<64, T>, smem)) return ATTN_ERR_LAUNCH;
-    exattn::attn_fwd_kernel<64, T><<<grid, exattn::FwdCfg<64>::kThreads, smem, s>>>(p);
-  } else {
-    constexpr int smem = exattn::FwdCfg<128>::kSmem;
+  if constexpr (sizeof(T) == 1) {  // e4m3: head_dim 128 only
+    if (d != 128) return ATTN_ERR_INVALID;
+    constexpr int smem = exattn::FwdCfg<128, T>::kSmem;
     if (!ensure_smem_attr(exattn::attn_fwd_kernel<128, T>, smem)) return ATTN_ERR_LAUNCH;
-    exattn::attn_fwd_kernel<128, T><<<grid, exattn::FwdCfg<128>::kThreads, smem, s>>>(p);
+    exattn::attn_fwd_kernel<128, T><<<grid, exattn::FwdCfg<128, T>::kThreads, smem, s>>>(p);
+  } else if (d == 64) {
+    constexpr int smem = exattn::FwdCfg<64, T>::kSmem;
+    if (!ensure_smem_attr(exattn::attn_fwd_kernel<64, T>, smem)) return ATTN_ERR_LAUNCH;
+    exattn::attn_fwd_kernel<64, T><<<grid, exattn::FwdCfg<64, T>::kThreads, smem, s>>>(p);
+  } else {
+    constexpr int smem = exattn::FwdCfg<128, T>::kSmem;
+    if (!ensure_smem_attr(exattn::attn_fwd_kernel<128, T>, smem)) return ATTN_ERR_LAUNCH;
+    exattn::attn_fwd_kernel<128, T><<<grid, exattn::FwdCfg<128, T>::kThreads, smem, s>>>(p);
   }
   return launch_status();
 }
@@ -221,7 +229,46 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.causal = causal ? 1 : 0;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.o_mul = 1.0f;
   return launch_fwd<T>(p, d, dev, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// e4m3 inputs: the per-tensor descale factors fold into the score scale (Q,
+// K) and the output factor (V).
+int fwd_fp8_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                 float scale, int causal, float q_descale, float k_descale, float v_descale, attn_stream_t stream) {
+  const int sz = check_sizes(B, H, N, d);
+  if (sz < 0 || !check_scale(scale) || d != 128) return ATTN_ERR_INVALID;
+  if (!check_scale(q_descale) || !check_scale(k_descale) || !check_scale(v_descale)) return ATTN_ERR_INVALID;
+  const float eff = scale * q_descale * k_descale;
+  if (!check_scale(eff)) return ATTN_ERR_INVALID;
+  if (sz == 1) return ATTN_OK;
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return ATTN_ERR_INVALID;
+  int dev = 0;
+  if (int st = check_device(&dev)) return st;
+  FwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  const int BH = B * H;
+  if (!make_map_16<__nv_fp8_e4m3>(&p.tm_q, q, BH, N, d) || !make_map_16<__nv_fp8_e4m3>(&p.tm_k, k, BH, N, d) ||
+      !make_map_16<__nv_fp8_e4m3>(&p.tm_v, v, BH, N, d))
+    return ATTN_ERR_LAUNCH;
+  p.o = o;
+  p.lse = lse;
+  p.N = N;
+  p.Nk = N;
+  p.q_off = 0;
+  p.BH = BH;
+  p.nblocks = (N + 255) / 256;
+  p.splits = 1;
+  p.tps = (N + 127) / 128;
+  p.head_group = head_group(BH, 2.0 * N * d);  // K and V of one head
+  p.causal = causal ? 1 : 0;
+  p.scale = eff;
+  p.scale_log2 = eff * 1.4426950408889634f;
+  p.o_mul = v_descale;
+  return launch_fwd<__nv_fp8_e4m3>(p, d, dev, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // ------------------------------------------------------ split-key forward
@@ -367,6 +414,7 @@ int kvsplit_impl(const void* q, const void* k, const void* v, void* o, float* ls
   p.causal = causal ? 1 : 0;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.o_mul = 1.0f;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (int st = launch_fwd<T>(p, d, dev, s)) return st;
   if (S == 1) return ATTN_OK;
@@ -543,6 +591,12 @@ int attn_fwd_kvsplit(const void* q, const void* k, const void* v, void* o, float
                      size_t workspace_bytes_given, attn_stream_t stream) {
   return kvsplit_impl<__nv_bfloat16>(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, splits, workspace,
                                      workspace_bytes_given, stream);
+}
+
+// ------------------------------------------------------------- e4m3 forward
+int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                 float scale, int causal, float q_descale, float k_descale, float v_descale, attn_stream_t stream) {
+  return fwd_fp8_impl(q, k, v, o, lse, B, H, N, d, scale, causal, q_descale, k_descale, v_descale, stream);
 }
 
 // ------------------------------------------------------------- fp16 entry points

@@ -43,8 +43,9 @@ struct FwdParams {
   float* part_lse;  // splits > 1: [B*H, splits, N] fp32 partial LSE (-inf where the range saw no key)
   int head_group;  // heads whose CTAs are scheduled together (L2 reuse of K/V)
   int causal;
-  float scale;       // softmax scale
+  float scale;       // softmax scale (times the Q and K descale factors for e4m3 inputs)
   float scale_log2;  // scale * log2(e)
+  float o_mul;       // factor applied to O on output (the V descale factor for e4m3 inputs, else 1)
   unsigned long long timeout_ns;
   unsigned int debug_flags;
 };
@@ -54,21 +55,31 @@ struct FwdParams {
 // d = 128 (one exp per score against 4*d flops of MMA).
 constexpr int kEmuPairs = 3;
 
-template <int D>
+// T: the input element type (16-bit, or e4m3).  A tile row holds D
+// elements; tiles are stored as 128-byte swizzled chunks of 128 rows.
+template <int D, typename T>
 struct FwdCfg {
   static constexpr int kThreads = 320;  // 8 softmax warps, producer warp, MMA warp
-  static constexpr uint32_t kTile = 128u * D * 2u;  // one 128-row bf16 tile
-  static constexpr int kSlots = (D == 128) ? 4 : 8;  // K/V ring slots
-  static constexpr int kChunks = D / 64;             // 64-column swizzle chunks per tile
+  static constexpr uint32_t kElem = sizeof(T);
+  static constexpr uint32_t kTile = 128u * D * kElem;          // one 128-row tile
+  static constexpr int kSlots = (kTile == 32768u) ? 4 : 8;     // K/V ring slots
+  static constexpr int kChunks = D * kElem / 128;              // 128-byte swizzle chunks per row
+  static constexpr int kChunkElems = 128 / kElem;              // elements per chunk
+  static constexpr int kKStep = 32 / kElem;                    // K of one MMA (32 bytes of a row)
+  static constexpr int kSSteps = D / kKStep;                   // MMAs of one S product
+  static constexpr int kPVSteps = 128 / kKStep;                // MMAs of one P V product (128 keys)
+  static constexpr int kPCols = 128 * kElem / 4;               // TMEM columns of P (128 keys)
   static constexpr uint32_t kBarOff = (2 + kSlots) * kTile;
   static constexpr uint32_t kSmem = kBarOff + 256;
 };
 
-// T: the 16-bit element type of Q, K, V and O (__nv_bfloat16 or __half).
+// T: the element type of Q, K and V (__nv_bfloat16, __half, or __nv_fp8_e4m3);
+// O has type Elem<T>::Out.
 template <int D, typename T>
-__global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1) attn_fwd_kernel(const __grid_constant__ FwdParams p) {
-  using C = FwdCfg<D>;
+__global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, 1) attn_fwd_kernel(const __grid_constant__ FwdParams p) {
+  using C = FwdCfg<D, T>;
   using E = Elem<T>;
+  using TO = typename E::Out;
   constexpr int kProducerWarp = 8;
   constexpr int kMmaWarp = 9;
   constexpr int SLOTS = C::kSlots;
@@ -153,8 +164,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1) attn_fwd_kernel(const 
       mbar_arrive_expect_tx(bar_q, TILE * (n_sub[1] > 0 ? 2u : 1u));
 #pragma unroll
       for (int c = 0; c < C::kChunks; ++c) {
-        tma_load_3d(sQ + c * 16384, &p.tm_q, bar_q, c * 64, qb * 256, bh);
-        if (n_sub[1] > 0) tma_load_3d(sQ + TILE + c * 16384, &p.tm_q, bar_q, c * 64, qb * 256 + 128, bh);
+        tma_load_3d(sQ + c * 16384, &p.tm_q, bar_q, c * C::kChunkElems, qb * 256, bh);
+        if (n_sub[1] > 0)
+          tma_load_3d(sQ + TILE + c * 16384, &p.tm_q, bar_q, c * C::kChunkElems, qb * 256 + 128, bh);
       }
       int last_par[SLOTS];
 #pragma unroll
@@ -175,7 +187,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1) attn_fwd_kernel(const 
           const CUtensorMap* m = x ? &p.tm_v : &p.tm_k;
 #pragma unroll
           for (int c = 0; c < C::kChunks; ++c)
-            tma_load_3d(sKV + slot * TILE + c * 16384, m, &bar_full[slot], c * 64, (j0 + j) * 128, bh);
+            tma_load_3d(sKV + slot * TILE + c * 16384, m, &bar_full[slot], c * C::kChunkElems, (j0 + j) * 128, bh);
 #pragma unroll
           for (int s = 0; s < SLOTS; ++s)
             if (s == slot) last_par[s] = static_cast<int>(ph);
@@ -211,18 +223,26 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1) attn_fwd_kernel(const 
         const uint32_t b0 = (skv0 - sq0) + slot * TILE;  // K_j, relative to sQ
         const uint32_t dt = tmem + k * 256;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(dt, desc_at(dK, a0 + off), desc_at(dK, b0 + off), idesc_s, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < C::kSSteps; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;  // 32 bytes of each row per MMA
+          if constexpr (E::kF8)
+            mma_ss_f8(dt, desc_at(dK, a0 + off), desc_at(dK, b0 + off), idesc_s, kk > 0 ? 1u : 0u);
+          else
+            mma_ss(dt, desc_at(dK, a0 + off), desc_at(dK, b0 + off), idesc_s, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int k, int slot, bool acc) {
         const uint32_t b0 = slot * TILE;  // V_j, relative to the ring
         const uint32_t dt = tmem + k * 256 + 128;
         const uint32_t at = tmem + k * 256;
+        // each MMA takes kKStep keys: 8 TMEM columns of P, kKStep 128-byte rows of V
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(dt, at + kk * 8, desc_at(dMN, b0 + kk * 2048), idesc_o, (acc || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < C::kPVSteps; ++kk) {
+          if constexpr (E::kF8)
+            mma_ts_f8(dt, at + kk * 8, desc_at(dMN, b0 + kk * C::kKStep * 128), idesc_o, (acc || kk > 0) ? 1u : 0u);
+          else
+            mma_ts(dt, at + kk * 8, desc_at(dMN, b0 + kk * C::kKStep * 128), idesc_o, (acc || kk > 0) ? 1u : 0u);
+        }
       };
       const int n0 = n_sub[0], n1 = n_sub[1];
       bool ok = mbar_wait(bar_q, 0, abort_flag, tmo, 110);
@@ -281,7 +301,15 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1) attn_fwd_kernel(const 
     const int row = wq * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const float c = p.scale_log2;
-    const float thr = 8.0f / c;  // reference max moves only if exps would exceed 2^8
+    // The reference max moves only if exps would exceed 2^kLazy.  For e4m3
+    // probabilities the limit is 2^2 and every P is scaled by 2^6 before it
+    // is rounded, so that P stays in [0, 256] (inside e4m3's range, 448) and
+    // all but negligible probabilities keep e4m3's full 3-bit precision
+    // instead of falling to its subnormals; l carries the same factor, which
+    // cancels in O / l and is taken out of the LSE.
+    constexpr float kLazy = E::kF8 ? 2.0f : 8.0f;
+    constexpr float kPLog2 = E::kF8 ? 6.0f : 0.0f;
+    const float thr = kLazy / c;
 
     // One step of the online softmax for sub-tile k, key tile j: load S_k,
     // mask, move the reference maximum if needed (rescaling O_k), write P_k
@@ -322,9 +350,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1) attn_fwd_kernel(const 
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
       const float alpha = ex2((m_ref - m_use) * c);
       const uint64_t c2 = f2_pack(c, c);
-      const uint64_t neg2 = f2_pack(-m_use * c, -m_use * c);
+      const uint64_t neg2 = f2_pack(kPLog2 - m_use * c, kPLog2 - m_use * c);
       uint64_t suma[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
-      uint32_t pk[64];
+      uint32_t pk[64];  // 16-bit: one pair of keys per word; e4m3: words 0..31, four keys each
+      uint64_t pk2_prev = 0;  // e4m3: the even pair, held until the odd one completes a word
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
         const uint64_t x = f2_fma(f2_pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), c2, neg2);
@@ -339,14 +368,25 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1) attn_fwd_kernel(const 
         suma[i & 1] = f2_add(suma[i & 1], pp);
         float p0, p1;
         f2_unpack(pp, p0, p1);
-        pk[i] = E::pack2(p0, p1);
+        if constexpr (E::kF8) {
+          if (i & 1) {
+            float q0, q1;
+            f2_unpack(pk2_prev, q0, q1);
+            pk[i >> 1] = E::pack4(q0, q1, p0, p1);
+          } else {
+            pk2_prev = pp;
+          }
+        } else {
+          pk[i] = E::pack2(p0, p1);
+        }
       }
       float s0, s1, s2, s3;
       f2_unpack(suma[0], s0, s1);
       f2_unpack(suma[1], s2, s3);
       l = l * alpha + ((s0 + s1) + (s2 + s3));
 #pragma unroll
-      for (int i = 0; i < 4; ++i) tmem_st16(tS + 16 * i, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * i]));
+      for (int i = 0; i < C::kPCols / 16; ++i)
+        tmem_st16(tS + 16 * i, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * i]));
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
@@ -375,7 +415,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1) attn_fwd_kernel(const 
       if (p.part_o != nullptr) {
         // one key range of a split row: O normalised by this range's own sum,
         // and the range's logsumexp (-inf if the row saw none of its keys)
-        const float inv_l = l > 0.f ? 1.0f / l : 0.f;
+        const float inv_l = l > 0.f ? p.o_mul / l : 0.f;
         const size_t prow = (static_cast<size_t>(bh) * p.splits + split) * N + q_row;
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
@@ -390,11 +430,11 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1) attn_fwd_kernel(const 
                                    __uint_as_float(o[4 * i + 2]) * inv_l, __uint_as_float(o[4 * i + 3]) * inv_l);
           }
         }
-        if (q_row < N) p.part_lse[prow] = l > 0.f ? m_ref * p.scale + __logf(l) : -INFINITY;
+        if (q_row < N) p.part_lse[prow] = l > 0.f ? m_ref * p.scale + __logf(l) - kPLog2 * 0.6931471805599453f : -INFINITY;
         return;
       }
-      const float inv_l = 1.0f / l;
-      T* orow = static_cast<T*>(p.o) + (static_cast<size_t>(bh) * N + q_row) * D;
+      const float inv_l = p.o_mul / l;
+      TO* orow = static_cast<TO*>(p.o) + (static_cast<size_t>(bh) * N + q_row) * D;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
@@ -404,13 +444,14 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1) attn_fwd_kernel(const 
           uint32_t w[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            w[i] = E::pack2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+            w[i] = Elem<TO>::pack2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
           uint4* dst = reinterpret_cast<uint4*>(orow + 32 * cc);
 #pragma unroll
           for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
         }
       }
-      if (q_row < N) p.lse[static_cast<size_t>(bh) * N + q_row] = m_ref * p.scale + __logf(l);
+      if (q_row < N)
+        p.lse[static_cast<size_t>(bh) * N + q_row] = m_ref * p.scale + __logf(l) - kPLog2 * 0.6931471805599453f;
     };
 
     const int k = warp >> 2;  // sub-tile

@@ -10,6 +10,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 namespace exattn {
 
@@ -199,9 +200,27 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
-// Instruction descriptor, kind::f16 with 16-bit A/B (fp16: format 0, bf16:
-// format 1; both operands of one MMA have the same type) and fp32
-// accumulate.  a_mn / b_mn: 0 = K-major operand, 1 = MN-major operand.
+// The same two forms for kind::f8f6f4 (8-bit A and B, fp32 accumulate).
+// The four zero words are the disable-output-lane mask (no lane disabled).
+__device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u));
+}
+__device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u));
+}
+
+// Instruction descriptor with fp32 accumulate.  kind::f16: A/B format 0 =
+// fp16, 1 = bf16 (both operands of one MMA have the same type); kind::f8f6f4:
+// format 0 = e4m3.  a_mn / b_mn: 0 = K-major operand, 1 = MN-major operand
+// (MN-major is allowed for the 16-bit and the 8-bit e4m3/e5m2 formats).
 __host__ __device__ constexpr uint32_t idesc_16_f32(uint32_t ab_fmt, int M, int N, int a_mn, int b_mn) {
   return (1u << 4)                          // D format: f32
          | (ab_fmt << 7)                    // A format
@@ -446,6 +465,8 @@ template <typename T>
 struct Elem;
 template <>
 struct Elem<__nv_bfloat16> {
+  using Out = __nv_bfloat16;  // output element type of a forward on this input type
+  static constexpr bool kF8 = false;
   static constexpr uint32_t kMmaFmt = 1;
   __device__ static __forceinline__ uint32_t pack2(float lo, float hi) { return pack_bf16x2(lo, hi); }
   __device__ static __forceinline__ float2 unpack2(uint32_t w) {
@@ -454,10 +475,26 @@ struct Elem<__nv_bfloat16> {
 };
 template <>
 struct Elem<__half> {
+  using Out = __half;
+  static constexpr bool kF8 = false;
   static constexpr uint32_t kMmaFmt = 0;
   __device__ static __forceinline__ uint32_t pack2(float lo, float hi) { return pack_f16x2(lo, hi); }
   __device__ static __forceinline__ float2 unpack2(uint32_t w) {
     return __half22float2(*reinterpret_cast<const __half2*>(&w));
+  }
+};
+// e4m3 inputs (a forward only): kind::f8f6f4 operands, bf16 outputs.  pack4
+// rounds four fp32 values to nearest e4m3 (saturating at +-448), the first
+// in the lowest byte: four consecutive keys in one 32-bit TMEM column.
+template <>
+struct Elem<__nv_fp8_e4m3> {
+  using Out = __nv_bfloat16;
+  static constexpr bool kF8 = true;
+  static constexpr uint32_t kMmaFmt = 0;
+  __device__ static __forceinline__ uint32_t pack4(float a, float b, float c, float d) {
+    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+    const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+    return lo | (hi << 16);
   }
 };
 

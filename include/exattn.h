@@ -126,6 +126,26 @@ int attn_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, const
                         size_t workspace_bytes, attn_stream_t stream);
 
 /*
+ * Forward on FP8 (e4m3) inputs, the low-precision mode the pages give the
+ * third version of the method ("11.11 Flash Attention", section "Flash
+ * Attention 3", FP8 support; the v1/v2/v3 comparison table of "Walk through
+ * the FlashAttention algorithm ...").
+ *   q, k, v : in,  e4m3 [B,H,N,d] (one byte per element), d = 128 only;
+ *             the real values are q * q_descale, k * k_descale, v * v_descale
+ *             (per-tensor factors, finite and > 0)
+ *   o       : out, bf16 [B,H,N,d]
+ *   lse     : out, fp32 [B,H,N], as attn_fwd, of the scaled real scores
+ * S = (scale q_descale k_descale) Q K^T is computed by e4m3 tensor-core
+ * products with fp32 accumulation.  The probabilities are scaled into e4m3's
+ * normal range and rounded to e4m3 for the P V product (relative error at
+ * most 2^-4 each); the softmax sums and the LSE use them unrounded, in fp32.
+ * Same conventions and status codes as attn_fwd (d != 128 is
+ * ATTN_ERR_INVALID).
+ */
+int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                 float scale, int causal, float q_descale, float k_descale, float v_descale, attn_stream_t stream);
+
+/*
  * Forward with the keys of each query row split into ranges: decode (a few
  * new queries against a long key/value history) and long rows that leave the
  * machine under-filled.
