@@ -423,10 +423,36 @@ def run_sweep(args):
                "burst_peak": burst, "peak_source": peak_src, "clocks": clk}
         rows.append(row)
         print(json.dumps(row), flush=True)
-    for row in kvsplit_points(dev, flush, burst, peak_src, args, only) + fp8_points(dev, flush, burst, args, only):
+    for row in (kvsplit_points(dev, flush, burst, peak_src, args, only) + fp8_points(dev, flush, burst, args, only)
+                + hdim256_points(dev, flush, burst, args, only)):
         rows.append(row)
         print(json.dumps(row), flush=True)
     return rows
+
+
+def hdim256_points(dev, flush, burst, args, only):
+    """The forward at head_dim 256 (one 128-row sub-tile per CTA)."""
+    import exact_attention_106_b200 as ex
+    from exact_attention_106_b200 import workloads as W
+    out = []
+    for w in W.HDIM256:
+        if only and w.name not in only:
+            continue
+        q, k, v, _ = (x.to(dev) if x is not None else None for x in W.make_inputs(w, with_grad_out=False))
+        o = torch.empty_like(q)
+        lse = torch.empty(w.shape[:3], dtype=torch.float32, device=dev)
+        med, mn, reps, clk = time_fn(lambda: ex.forward(q, k, v, causal=w.causal, scale=w.softmax_scale, out=o,
+                                                       lse=lse), dev, flush, args.sweep_reps, args.sweep_seconds)
+        tf = w.fwd_flops() / (med * 1e-3) / 1e12
+        mhz = clk["sm_mhz"] if clk else None
+        out.append({"point": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "reps": reps,
+                    "fwd_ms": med, "fwd_min_ms": mn, "fwd_tflops": tf, "fwd_of_burst": tf / burst,
+                    "fwd_of_spec_2250": tf / SPEC_PEAK_TFLOPS,
+                    "fwd_of_clock_peak": tf / (SM_COUNT * FLOP_PER_SM_CYCLE * mhz * 1e-6) if mhz else None,
+                    "clocks": clk})
+        del q, k, v, o, lse
+        torch.cuda.empty_cache()
+    return out
 
 
 def fp8_points(dev, flush, burst, args, only):

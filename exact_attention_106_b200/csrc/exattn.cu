@@ -47,6 +47,22 @@ int check_sizes(int B, int H, int N, int d) {
 
 bool check_scale(float scale) { return std::isfinite(scale) && scale > 0.f; }
 
+// Query rows per forward CTA: two 128-row sub-tiles, one at head_dim 256.
+int fwd_rows(int d) { return d == 256 ? 128 : 256; }
+
+// The forward also takes head_dim 256 (the backward does not).
+int check_sizes_fwd(int B, int H, int N, int d) {
+  if (d == 256) {
+    if (B < 0 || H < 0 || N < 0) return -1;
+    if (B == 0 || H == 0 || N == 0) return 1;
+    const long long bh = static_cast<long long>(B) * H;
+    if (bh > 0x7fffffffLL) return -1;
+    if ((static_cast<long long>(N) + 127) / 128 * bh > 0x7fffffffLL) return -1;
+    return 0;
+  }
+  return check_sizes(B, H, N, d);
+}
+
 size_t padded_rows(int N) { return (static_cast<size_t>(N) + 127) / 128 * 128; }
 
 struct Workspace {
@@ -186,6 +202,10 @@ int launch_fwd(FwdParams& p, int d, int dev, cudaStream_t s) {
     constexpr int smem = exattn::FwdCfg<128, T>::kSmem;
     if (!ensure_smem_attr(exattn::attn_fwd_kernel<128, T>, smem)) return ATTN_ERR_LAUNCH;
     exattn::attn_fwd_kernel<128, T><<<grid, exattn::FwdCfg<128, T>::kThreads, smem, s>>>(p);
+  } else if (d == 256) {
+    constexpr int smem = exattn::FwdCfg<256, T>::kSmem;
+    if (!ensure_smem_attr(exattn::attn_fwd_kernel<256, T>, smem)) return ATTN_ERR_LAUNCH;
+    exattn::attn_fwd_kernel<256, T><<<grid, exattn::FwdCfg<256, T>::kThreads, smem, s>>>(p);
   } else if (d == 64) {
     constexpr int smem = exattn::FwdCfg<64, T>::kSmem;
     if (!ensure_smem_attr(exattn::attn_fwd_kernel<64, T>, smem)) return ATTN_ERR_LAUNCH;
@@ -201,7 +221,7 @@ int launch_fwd(FwdParams& p, int d, int dev, cudaStream_t s) {
 template <typename T>
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
              float scale, int causal, attn_stream_t stream) {
-  const int sz = check_sizes(B, H, N, d);
+  const int sz = check_sizes_fwd(B, H, N, d);
   if (sz < 0 || !check_scale(scale)) return ATTN_ERR_INVALID;
   if (sz == 1) return ATTN_OK;
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID;
@@ -222,7 +242,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.Nk = N;
   p.q_off = 0;
   p.BH = BH;
-  p.nblocks = (N + 255) / 256;
+  p.nblocks = (N + fwd_rows(d) - 1) / fwd_rows(d);
   p.splits = 1;
   p.tps = (N + 127) / 128;
   p.head_group = head_group(BH, 2.0 * N * d * 2);  // K and V of one head
@@ -284,9 +304,9 @@ int sm_count() {
 
 // Key tiles that query block qb (256 rows) sees: all of them, or under the
 // causal mask those up to the last visible key of its last row.
-int block_tiles(int qb, int Nq, int Nk, int causal) {
+int block_tiles(int qb, int rows, int Nq, int Nk, int causal) {
   const int ntk = (Nk + 127) / 128;
-  const int last = std::min(qb * 256 + 255, Nq - 1);
+  const int last = std::min(qb * rows + rows - 1, Nq - 1);
   return causal ? std::min(ntk, (last + (Nk - Nq)) / 128 + 1) : ntk;
 }
 
@@ -297,14 +317,14 @@ int block_tiles(int qb, int Nq, int Nk, int causal) {
 // costing its key tiles plus a fixed start-up cost, and S > 1 pays for the
 // merge pass; the S with the shortest makespan wins.  The result depends only
 // on the sizes and the SM count and is cached.
-int choose_splits(int BH, int Nq, int Nk, int causal) {
+int choose_splits(int BH, int Nq, int Nk, int causal, int rows) {
   const int sms = sm_count();
-  const int nblocks = (Nq + 255) / 256;
+  const int nblocks = (Nq + rows - 1) / rows;
   const int ntk = (Nk + 127) / 128;
   if (static_cast<long long>(BH) * nblocks >= 4LL * sms || ntk == 1) return 1;
   static std::mutex mu;
-  static std::map<std::tuple<int, int, int, int, int>, int> cache;
-  const auto key = std::make_tuple(BH, Nq, Nk, causal, sms);
+  static std::map<std::tuple<int, int, int, int, int, int>, int> cache;
+  const auto key = std::make_tuple(BH, Nq, Nk, causal, sms, rows);
   {
     std::lock_guard<std::mutex> lock(mu);
     auto it = cache.find(key);
@@ -323,7 +343,7 @@ int choose_splits(int BH, int Nq, int Nk, int causal) {
     double makespan = 0;
     for (int r = 0; r < nblocks * S; ++r) {
       const int qb = nblocks - 1 - r / S, sp = r % S;
-      const int cnt = std::max(0, std::min(block_tiles(qb, Nq, Nk, causal) - sp * tps, tps));
+      const int cnt = std::max(0, std::min(block_tiles(qb, rows, Nq, Nk, causal) - sp * tps, tps));
       for (int h = 0; h < BH; ++h) {
         const double t = free_at.top() + cnt + kStartup;
         free_at.pop();
@@ -344,9 +364,9 @@ int choose_splits(int BH, int Nq, int Nk, int causal) {
 }
 
 // Resolves the split count (0 = automatic) and the key tiles per range.
-void resolve_splits(int BH, int Nq, int Nk, int causal, int requested, int* splits, int* tps) {
+void resolve_splits(int BH, int Nq, int Nk, int d, int causal, int requested, int* splits, int* tps) {
   const int ntk = (Nk + 127) / 128;
-  int S = requested > 0 ? std::min(requested, kMaxSplits) : choose_splits(BH, Nq, Nk, causal);
+  int S = requested > 0 ? std::min(requested, kMaxSplits) : choose_splits(BH, Nq, Nk, causal, fwd_rows(d));
   S = std::max(1, std::min(S, ntk));
   const int t = (ntk + S - 1) / S;
   *tps = t;
@@ -363,11 +383,11 @@ size_t kvsplit_ws_bytes(int BH, int Nq, int d, int S) {
 
 int check_kvsplit_sizes(int B, int H, int Nq, int Nk, int d, int causal, int splits) {
   if (Nk < 0 || splits < 0) return -1;
-  const int sz = check_sizes(B, H, Nq, d);
+  const int sz = check_sizes_fwd(B, H, Nq, d);
   if (sz != 0) return sz;
   if (Nk == 0) return -1;             // a query with no keys has no softmax
   if (causal && Nq > Nk) return -1;  // the first rows would see no key
-  const long long units = static_cast<long long>(B) * H * ((Nq + 255) / 256) * kMaxSplits;
+  const long long units = static_cast<long long>(B) * H * ((Nq + 127) / 128) * kMaxSplits;
   if (units > 0x7fffffffLL) return -1;
   return 0;
 }
@@ -386,7 +406,7 @@ int kvsplit_impl(const void* q, const void* k, const void* v, void* o, float* ls
   if (int st = check_device(&dev)) return st;
   const int BH = B * H;
   int S = 1, tps = 1;
-  resolve_splits(BH, Nq, Nk, causal ? 1 : 0, splits, &S, &tps);
+  resolve_splits(BH, Nq, Nk, d, causal ? 1 : 0, splits, &S, &tps);
   const size_t need = kvsplit_ws_bytes(BH, Nq, d, S);
   if (need > 0 && (!workspace || workspace_bytes_given < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)))
     return ATTN_ERR_INVALID;
@@ -402,7 +422,7 @@ int kvsplit_impl(const void* q, const void* k, const void* v, void* o, float* ls
   p.Nk = Nk;
   p.q_off = Nk - Nq;
   p.BH = BH;
-  p.nblocks = (Nq + 255) / 256;
+  p.nblocks = (Nq + fwd_rows(d) - 1) / fwd_rows(d);
   p.splits = S;
   p.tps = tps;
   if (S > 1) {
@@ -422,8 +442,10 @@ int kvsplit_impl(const void* q, const void* k, const void* v, void* o, float* ls
   const unsigned blocks = static_cast<unsigned>((rows + 7) / 8);
   if (d == 64)
     exattn::attn_fwd_merge_kernel<64, T><<<blocks, 256, 0, s>>>(p.part_o, p.part_lse, o, lse, BH, Nq, S);
-  else
+  else if (d == 128)
     exattn::attn_fwd_merge_kernel<128, T><<<blocks, 256, 0, s>>>(p.part_o, p.part_lse, o, lse, BH, Nq, S);
+  else
+    exattn::attn_fwd_merge_kernel<256, T><<<blocks, 256, 0, s>>>(p.part_o, p.part_lse, o, lse, BH, Nq, S);
   return launch_status();
 }
 
@@ -575,14 +597,14 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
 size_t attn_fwd_kvsplit_workspace_bytes(int B, int H, int Nq, int Nk, int d, int causal, int splits) {
   if (check_kvsplit_sizes(B, H, Nq, Nk, d, causal, splits) != 0) return 0;
   int S = 1, tps = 1;
-  resolve_splits(B * H, Nq, Nk, causal ? 1 : 0, splits, &S, &tps);
+  resolve_splits(B * H, Nq, Nk, d, causal ? 1 : 0, splits, &S, &tps);
   return kvsplit_ws_bytes(B * H, Nq, d, S);
 }
 
 int attn_fwd_kvsplit_count(int B, int H, int Nq, int Nk, int d, int causal, int splits) {
   if (check_kvsplit_sizes(B, H, Nq, Nk, d, causal, splits) != 0) return 0;
   int S = 1, tps = 1;
-  resolve_splits(B * H, Nq, Nk, causal ? 1 : 0, splits, &S, &tps);
+  resolve_splits(B * H, Nq, Nk, d, causal ? 1 : 0, splits, &S, &tps);
   return S;
 }
 

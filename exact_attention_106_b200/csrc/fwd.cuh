@@ -6,7 +6,9 @@
 //
 // One CTA owns a 256-row block of queries of one (batch, head), split into two
 // 128-row sub-tiles that ping-pong on the tensor core (while the softmax of
-// one sub-tile runs, the MMAs of the other do).  Roles (320 threads):
+// one sub-tile runs, the MMAs of the other do).  At head_dim 256 a CTA owns one
+// 128-row sub-tile (warps 0..3 softmax, 4 producer, 5 MMA): its O accumulator
+// takes 256 TMEM columns.  Roles (320 threads):
 //   warps 0..3    softmax of sub-tile 0 (one thread per query row)
 //   warps 4..7    softmax of sub-tile 1
 //   warp 8        TMA producer: Q (once), then K_j and V_j into a smem ring
@@ -14,7 +16,7 @@
 // Tensor memory (512 columns x 128 lanes of 32 bit), per sub-tile k:
 //   columns [256k, 256k+128)      S_k = Q_k K_j^T (fp32); P_k (16-bit pairs) is
 //                                 written back over its first 64 columns
-//   columns [256k+128, +d)        O_k accumulator (fp32)
+//   columns [256k+128, +d)        O_k accumulator (fp32; d = 256: columns 128..383)
 // The softmax keeps, per row, a reference maximum and the running sum l;
 // the division by l happens once at the end (section "Flash Attention 2":
 // fewer non-matmul operations).  The reference maximum only moves when a
@@ -59,17 +61,23 @@ constexpr int kEmuPairs = 3;
 // elements; tiles are stored as 128-byte swizzled chunks of 128 rows.
 template <int D, typename T>
 struct FwdCfg {
-  static constexpr int kThreads = 320;  // 8 softmax warps, producer warp, MMA warp
+  // 128-row query sub-tiles per CTA: two, except at head_dim 256, where one
+  // sub-tile's S (128 columns) and O (256) already take 384 of the 512 TMEM
+  // columns.
+  static constexpr int kSub = (D == 256) ? 1 : 2;
+  static constexpr int kRows = 128 * kSub;                     // query rows per CTA
+  static constexpr int kThreads = 128 * kSub + 64;             // softmax warps, producer warp, MMA warp
   static constexpr uint32_t kElem = sizeof(T);
   static constexpr uint32_t kTile = 128u * D * kElem;          // one 128-row tile
-  static constexpr int kSlots = (kTile == 32768u) ? 4 : 8;     // K/V ring slots
+  // K/V ring slots within the 227 KB of shared memory
+  static constexpr int kSlots = (kTile == 65536u) ? 2 : (kTile == 32768u) ? 4 : 8;
   static constexpr int kChunks = D * kElem / 128;              // 128-byte swizzle chunks per row
   static constexpr int kChunkElems = 128 / kElem;              // elements per chunk
   static constexpr int kKStep = 32 / kElem;                    // K of one MMA (32 bytes of a row)
   static constexpr int kSSteps = D / kKStep;                   // MMAs of one S product
   static constexpr int kPVSteps = 128 / kKStep;                // MMAs of one P V product (128 keys)
   static constexpr int kPCols = 128 * kElem / 4;               // TMEM columns of P (128 keys)
-  static constexpr uint32_t kBarOff = (2 + kSlots) * kTile;
+  static constexpr uint32_t kBarOff = (kSub + kSlots) * kTile;
   static constexpr uint32_t kSmem = kBarOff + 256;
 };
 
@@ -80,8 +88,9 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, 1) attn_fwd_kernel(con
   using C = FwdCfg<D, T>;
   using E = Elem<T>;
   using TO = typename E::Out;
-  constexpr int kProducerWarp = 8;
-  constexpr int kMmaWarp = 9;
+  constexpr int kProducerWarp = 4 * C::kSub;
+  constexpr int kMmaWarp = kProducerWarp + 1;
+  constexpr int RW = C::kRows;
   constexpr int SLOTS = C::kSlots;
   constexpr uint32_t TILE = C::kTile;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -91,7 +100,7 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, 1) attn_fwd_kernel(con
     return;
   }
   uint8_t* sQ = smem;
-  uint8_t* sKV = smem + 2 * TILE;
+  uint8_t* sKV = smem + C::kSub * TILE;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint64_t* bar_q = bars;
   uint64_t* bar_full = bars + 1;
@@ -120,9 +129,9 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, 1) attn_fwd_kernel(con
   int n_sub[2];
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
-    const int row0 = qb * 256 + k * 128;
+    const int row0 = qb * RW + k * 128;
     int n = 0;
-    if (row0 < N) {
+    if (k < C::kSub && row0 < N) {
       const int last = min(row0 + 127, N - 1);
       n = p.causal ? min(ntk, (last + p.q_off) / 128 + 1) : ntk;
     }
@@ -164,9 +173,9 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, 1) attn_fwd_kernel(con
       mbar_arrive_expect_tx(bar_q, TILE * (n_sub[1] > 0 ? 2u : 1u));
 #pragma unroll
       for (int c = 0; c < C::kChunks; ++c) {
-        tma_load_3d(sQ + c * 16384, &p.tm_q, bar_q, c * C::kChunkElems, qb * 256, bh);
+        tma_load_3d(sQ + c * 16384, &p.tm_q, bar_q, c * C::kChunkElems, qb * RW, bh);
         if (n_sub[1] > 0)
-          tma_load_3d(sQ + TILE + c * 16384, &p.tm_q, bar_q, c * C::kChunkElems, qb * 256 + 128, bh);
+          tma_load_3d(sQ + TILE + c * 16384, &p.tm_q, bar_q, c * C::kChunkElems, qb * RW + 128, bh);
       }
       int last_par[SLOTS];
 #pragma unroll
@@ -328,10 +337,10 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, 1) attn_fwd_kernel(con
       tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
       tmem_wait_ld();
       const int key0 = (j0 + j) * 128;
-      const int q_row = qb * 256 + k * 128 + row;
+      const int q_row = qb * RW + k * 128 + row;
       // masking is needed where the sub-tile's first row does not see the
       // whole tile, or on the ragged last key tile
-      const bool part = p.causal && key0 + 127 > qb * 256 + k * 128 + p.q_off;
+      const bool part = p.causal && key0 + 127 > qb * RW + k * 128 + p.q_off;
       if (part || key0 + 128 > Nk) {
         const int lim = min(part ? q_row + p.q_off - key0 : 127, Nk - 1 - key0);  // last visible column
 #pragma unroll
@@ -411,7 +420,7 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, 1) attn_fwd_kernel(con
       if (!__all_sync(0xffffffffu, mbar_wait(&bar_o[k], 0, abort_flag, tmo, 122 + k))) return;
       tc_fence_after();
       const uint32_t tO = lane_base + k * 256 + 128;
-      const int q_row = qb * 256 + k * 128 + row;
+      const int q_row = qb * RW + k * 128 + row;
       if (p.part_o != nullptr) {
         // one key range of a split row: O normalised by this range's own sum,
         // and the range's logsumexp (-inf if the row saw none of its keys)
@@ -462,7 +471,7 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, 1) attn_fwd_kernel(con
     if (ok && n > 0) epilogue(k, m_ref, l);
     if (n == 0 && p.part_o != nullptr) {
       // a range that holds none of this sub-tile's visible keys: an empty part
-      const int q_row = qb * 256 + k * 128 + row;
+      const int q_row = qb * RW + k * 128 + row;
       if (q_row < N) {
         const size_t prow = (static_cast<size_t>(bh) * p.splits + split) * N + q_row;
         float4* dst = reinterpret_cast<float4*>(p.part_o + prow * D);
@@ -509,12 +518,15 @@ __global__ void __launch_bounds__(256) attn_fwd_merge_kernel(const float* __rest
       const float w = __expf(part_lse[pr] - m);
       wsum += w;
       const float* src = part_o + pr * D + lane * V;
-      if constexpr (V == 4) {
-        const float4 x = *reinterpret_cast<const float4*>(src);
-        acc[0] += w * x.x;
-        acc[1] += w * x.y;
-        acc[2] += w * x.z;
-        acc[3] += w * x.w;
+      if constexpr (V >= 4) {
+#pragma unroll
+        for (int c4 = 0; c4 < V / 4; ++c4) {
+          const float4 x = reinterpret_cast<const float4*>(src)[c4];
+          acc[4 * c4] += w * x.x;
+          acc[4 * c4 + 1] += w * x.y;
+          acc[4 * c4 + 2] += w * x.z;
+          acc[4 * c4 + 3] += w * x.w;
+        }
       } else {
         const float2 x = *reinterpret_cast<const float2*>(src);
         acc[0] += w * x.x;
@@ -527,7 +539,9 @@ __global__ void __launch_bounds__(256) attn_fwd_merge_kernel(const float* __rest
 #pragma unroll
   for (int c = 0; c < V / 2; ++c) w2[c] = Elem<T>::pack2(acc[2 * c] * inv, acc[2 * c + 1] * inv);
   T* dst = static_cast<T*>(o) + row * D + lane * V;
-  if constexpr (V == 4)
+  if constexpr (V == 8)
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+  else if constexpr (V == 4)
     *reinterpret_cast<uint2*>(dst) = make_uint2(w2[0], w2[1]);
   else
     *reinterpret_cast<uint32_t*>(dst) = w2[0];

@@ -114,6 +114,11 @@ def sweep() -> List[Workload]:
     return out
 
 
+# head_dim 256, the largest the pages mention (PyTorch SDPA's limit, "11.11
+# Flash Attention", section "Using Flash Attention"); forward only.
+HDIM256 = [Workload("hdim256_2x16x8192x256_causal", 2, 16, 8192, 256, True, 8000),
+           Workload("hdim256_1x16x16384x256_full", 1, 16, 16384, 256, False, 8100)]
+
 SINGLE_HEAD_32K = Workload("single_head_1x1x32768x128_full", 1, 1, 32768, 128, False, 6000)
 SINGLE_HEAD_32K_CAUSAL = Workload("single_head_1x1x32768x128_causal", 1, 1, 32768, 128, True, 6100)
 
@@ -169,7 +174,7 @@ DECODES = [DECODE_1Q, DECODE_16Q]
 
 
 def by_name(name: str):
-    for w in NAMED + sweep() + [SINGLE_HEAD_32K, SINGLE_HEAD_32K_CAUSAL] + DECODES:
+    for w in NAMED + sweep() + [SINGLE_HEAD_32K, SINGLE_HEAD_32K_CAUSAL] + DECODES + HDIM256:
         if w.name == name:
             return w
     raise KeyError(name)
