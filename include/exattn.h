@@ -30,7 +30,10 @@
  *    patterns; the _fp16 entry points take fp16 instead), contiguous, row-major [B, H, N, d]: the (batch, heads,
  *    seq_len, head_dim) order of the pages' PyTorch examples.  lse is fp32
  *    [B, H, N].  All of them are DEVICE pointers on the current CUDA device.
- *  - d must be 64 or 128.  N >= 1 is arbitrary (no multiple-of-tile rule).
+ *  - d must be 64 or 128; the forward entry points (attn_fwd, attn_fwd_fp16,
+ *    attn_fwd_kvsplit) also take 256 (PyTorch SDPA's limit quoted in "11.11
+ *    Flash Attention", section "Using Flash Attention"); attn_fwd_fp8 takes
+ *    128 only.  N >= 1 is arbitrary (no multiple-of-tile rule).
  *    B, H or N equal to 0 is an empty problem: the call returns
  *    ATTN_OK and touches nothing (pointers may then be NULL).
  *  - causal != 0 applies the square top-left mask: query i sees key j iff
@@ -62,7 +65,7 @@ typedef struct CUstream_st* attn_stream_t;
 typedef enum attn_status {
   ATTN_OK = 0,
   ATTN_ERR_INVALID = 1,            /* bad argument: null/misaligned pointer, negative size,
-                                      d not in {64,128}, scale not finite or <= 0,
+                                      d not supported by the call, scale not finite or <= 0,
                                       workspace too small, size overflow */
   ATTN_ERR_UNSUPPORTED_DEVICE = 2, /* current device is not sm_100 (B200) */
   ATTN_ERR_LAUNCH = 3,             /* a CUDA call failed (launch, attribute, tensor map) */
@@ -157,7 +160,9 @@ int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* ls
  *           the square mask of attn_fwd).  Requires Nq <= Nk.
  *   splits: key ranges per query row; 0 lets the library choose (it simulates
  *           the launch on the device's SM count), n > 0 asks for n (capped at
- *           64 and at the number of 128-key tiles).
+ *           64 and at the number of 128-key tiles).  The ranges hold equal
+ *           numbers of tiles, ceil(tiles / n) each, so fewer than n may be
+ *           used (attn_fwd_kvsplit_count reports how many).
  *   workspace: device, 256-byte aligned, >= attn_fwd_kvsplit_workspace_bytes()
  *           with the same arguments (0 bytes, and NULL allowed, when a single
  *           range is used); contents on entry are ignored.

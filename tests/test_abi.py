@@ -51,7 +51,7 @@ def fwd(lib, **kw):
 
 
 @pytest.mark.parametrize("kw", [
-    dict(d=96), dict(d=256), dict(B=-1), dict(N=-5), dict(scale=0.0), dict(scale=-1.0),
+    dict(d=96), dict(d=32), dict(d=512), dict(B=-1), dict(N=-5), dict(scale=0.0), dict(scale=-1.0),
     dict(scale=float("inf")), dict(scale=float("nan")), dict(q=None), dict(lse=None),
     dict(k=P + 8), dict(o=P + 2),
 ])
@@ -68,6 +68,7 @@ def test_workspace_size(lib):
     assert lib.attn_bwd_workspace_bytes(1, 1, 1, 64) == (128 * 64 + 2 * 128) * 4
     assert lib.attn_bwd_workspace_bytes(2, 3, 129, 128) == 6 * (256 * 128 + 2 * 256) * 4
     assert lib.attn_bwd_workspace_bytes(1, 1, 8, 80) == 0
+    assert lib.attn_bwd_workspace_bytes(1, 1, 8, 256) == 0  # the backward takes d = 64, 128 only
     assert lib.attn_bwd_workspace_bytes(0, 1, 8, 64) == 0
 
 
@@ -80,6 +81,7 @@ def test_bwd_rejects_small_workspace_and_misalignment(lib):
     assert lib.attn_bwd_dkdv(P, P, P, P, P, P, 1, 2, 300, 128, 0.1, 1, P, 0, None) == _lib.ATTN_ERR_INVALID
     assert lib.attn_bwd_dq_convert(P, 1, 2, 300, 64, 0.0, P, need, None) == _lib.ATTN_ERR_INVALID
     assert lib.attn_bwd(*([P] * 9), 0, 2, 300, 128, 0.1, 1, None, 0, None) == _lib.ATTN_OK
+    assert lib.attn_bwd(*([P] * 9), 1, 2, 300, 256, 0.1, 1, P, 1 << 30, None) == _lib.ATTN_ERR_INVALID
 
 
 def _stage_bytes(G, N, d):
@@ -111,3 +113,34 @@ def test_host_call_rejects_bad_arguments(lib):
     assert lib.attn_fwd_bwd_host(*host, 1, 2, 300, 96, 0.1, 1, P, need, 1, None) == _lib.ATTN_ERR_INVALID
     assert lib.attn_fwd_bwd_host(*host, 1, 2, 300, 128, 0.0, 1, P, need, 1, None) == _lib.ATTN_ERR_INVALID
     assert lib.attn_fwd_bwd_host(*host, 1, 0, 300, 128, 0.1, 1, None, 0, 0, None) == _lib.ATTN_OK  # empty
+
+
+def test_kvsplit_and_fp8_reject_bad_arguments_on_host(lib):
+    v = _lib.ATTN_ERR_INVALID
+    # causal with more queries than keys; no keys; negative split count; d = 96
+    assert lib.attn_fwd_kvsplit(P, P, P, P, P, 1, 1, 20, 10, 64, 0.1, 1, 0, P, 1 << 20, None) == v
+    assert lib.attn_fwd_kvsplit(P, P, P, P, P, 1, 1, 20, 0, 64, 0.1, 0, 0, P, 1 << 20, None) == v
+    assert lib.attn_fwd_kvsplit(P, P, P, P, P, 1, 1, 20, 20, 64, 0.1, 0, -1, P, 1 << 20, None) == v
+    assert lib.attn_fwd_kvsplit(P, P, P, P, P, 1, 1, 20, 20, 96, 0.1, 0, 0, P, 1 << 20, None) == v
+    assert lib.attn_fwd_kvsplit_count(1, 1, 20, 10, 64, 1, 0) == 0
+    # e4m3: d must be 128, descale factors finite and > 0
+    assert lib.attn_fwd_fp8(P, P, P, P, P, 1, 1, 8, 64, 0.1, 0, 1.0, 1.0, 1.0, None) == v
+    assert lib.attn_fwd_fp8(P, P, P, P, P, 1, 1, 8, 128, 0.1, 0, 1.0, -1.0, 1.0, None) == v
+    # empty problems are a no-op
+    assert lib.attn_fwd_kvsplit(None, None, None, None, None, 1, 1, 0, 10, 64, 0.1, 0, 0, None, 0, None) == 0
+
+
+def test_kvsplit_plan_on_host(lib):
+    """The split count and workspace size need no GPU: one range (no
+    workspace) when (batch, head, block) CTAs fill four waves, and the
+    workspace holds (d + 1) fp32 per row and range, each part 256-aligned."""
+    assert lib.attn_fwd_kvsplit_count(4, 32, 8192, 8192, 128, 1, 0) == 1
+    assert lib.attn_fwd_kvsplit_workspace_bytes(4, 32, 8192, 8192, 128, 1, 0) == 0
+    S = lib.attn_fwd_kvsplit_count(1, 1, 32768, 32768, 128, 1, 0)
+    assert 2 <= S <= 64
+    rows = S * 32768
+    assert lib.attn_fwd_kvsplit_workspace_bytes(1, 1, 32768, 32768, 128, 1, 0) == \
+        (rows * 128 * 4 + 255) // 256 * 256 + (rows * 4 + 255) // 256 * 256
+    assert lib.attn_fwd_kvsplit_count(1, 1, 1000, 1000, 64, 0, 4) == 4
+    # 5 asked over 8 key tiles: ranges of ceil(8 / 5) = 2 tiles, so 4 of them
+    assert lib.attn_fwd_kvsplit_count(1, 1, 1000, 1000, 64, 0, 5) == 4

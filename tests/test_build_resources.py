@@ -65,9 +65,12 @@ def test_backward_register_split_fits(registers, d, elem):
     assert 32 * (2 * r + drain + side) <= 16384
 
 
-@pytest.mark.parametrize("elem", ELEMS)
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("elem,d", [(e, d) for e in ELEMS for d in (64, 128, 256)] + [("13__nv_fp8_e4m3", 128)])
 def test_forward_fits_the_sub_partitions(registers, d, elem):
     r = _kernel(registers, "attn_fwd_kernel", d, "FwdParams", elem)
-    per_sub = math.ceil(_const("fwd.cuh", "kThreads") // 32 / 4)
+    src = open(os.path.join(CSRC, "fwd.cuh")).read()
+    assert "static constexpr int kSub = (D == 256) ? 1 : 2;" in src
+    assert "static constexpr int kThreads = 128 * kSub + 64;" in src
+    threads = 128 * (1 if d == 256 else 2) + 64  # softmax warps per sub-tile, producer and MMA warps
+    per_sub = math.ceil(threads // 32 / 4)
     assert per_sub * 32 * r <= 16384, (r, per_sub)
