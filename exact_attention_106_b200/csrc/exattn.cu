@@ -218,6 +218,28 @@ int launch_fwd(FwdParams& p, int d, int dev, cudaStream_t s) {
   return launch_status();
 }
 
+// The lean configuration (one sub-tile, two CTAs per SM) for a split-key
+// forward with at most 128 query rows.
+template <typename T>
+int launch_fwd_lean(FwdParams& p, int d, cudaStream_t s) {
+  p.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
+  p.debug_flags = g_debug_flags.load(std::memory_order_relaxed);
+  const dim3 grid(static_cast<unsigned>(p.nblocks) * static_cast<unsigned>(p.splits) * static_cast<unsigned>(p.BH));
+  if (d == 64) {
+    using C = exattn::FwdCfg<64, T, true>;
+    if (!ensure_smem_attr(exattn::attn_fwd_kernel<64, T, true>, C::kSmem)) return ATTN_ERR_LAUNCH;
+    exattn::attn_fwd_kernel<64, T, true><<<grid, C::kThreads, C::kSmem, s>>>(p);
+  } else {
+    using C = exattn::FwdCfg<128, T, true>;
+    if (!ensure_smem_attr(exattn::attn_fwd_kernel<128, T, true>, C::kSmem)) return ATTN_ERR_LAUNCH;
+    exattn::attn_fwd_kernel<128, T, true><<<grid, C::kThreads, C::kSmem, s>>>(p);
+  }
+  return launch_status();
+}
+
+// Whether a split-key forward runs in the lean configuration.
+bool use_lean(int Nq, int d, int elem_bytes) { return Nq <= 128 && d <= 128 && elem_bytes == 2; }
+
 template <typename T>
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
              float scale, int causal, attn_stream_t stream) {
@@ -317,14 +339,14 @@ int block_tiles(int qb, int rows, int Nq, int Nk, int causal) {
 // costing its key tiles plus a fixed start-up cost, and S > 1 pays for the
 // merge pass; the S with the shortest makespan wins.  The result depends only
 // on the sizes and the SM count and is cached.
-int choose_splits(int BH, int Nq, int Nk, int causal, int rows) {
-  const int sms = sm_count();
+int choose_splits(int BH, int Nq, int Nk, int causal, int rows, int per_sm) {
+  const int sms = sm_count() * per_sm;  // CTAs resident at once
   const int nblocks = (Nq + rows - 1) / rows;
   const int ntk = (Nk + 127) / 128;
   if (static_cast<long long>(BH) * nblocks >= 4LL * sms || ntk == 1) return 1;
   static std::mutex mu;
   static std::map<std::tuple<int, int, int, int, int, int>, int> cache;
-  const auto key = std::make_tuple(BH, Nq, Nk, causal, sms, rows);
+  const auto key = std::make_tuple(BH, Nq, Nk, causal, sms, rows);  // sms counts resident CTAs
   {
     std::lock_guard<std::mutex> lock(mu);
     auto it = cache.find(key);
@@ -364,9 +386,12 @@ int choose_splits(int BH, int Nq, int Nk, int causal, int rows) {
 }
 
 // Resolves the split count (0 = automatic) and the key tiles per range.
-void resolve_splits(int BH, int Nq, int Nk, int d, int causal, int requested, int* splits, int* tps) {
+void resolve_splits(int BH, int Nq, int Nk, int d, int elem_bytes, int causal, int requested, int* splits,
+                    int* tps) {
   const int ntk = (Nk + 127) / 128;
-  int S = requested > 0 ? std::min(requested, kMaxSplits) : choose_splits(BH, Nq, Nk, causal, fwd_rows(d));
+  const bool lean = use_lean(Nq, d, elem_bytes);
+  int S = requested > 0 ? std::min(requested, kMaxSplits)
+                        : choose_splits(BH, Nq, Nk, causal, lean ? 128 : fwd_rows(d), lean ? 2 : 1);
   S = std::max(1, std::min(S, ntk));
   const int t = (ntk + S - 1) / S;
   *tps = t;
@@ -406,7 +431,7 @@ int kvsplit_impl(const void* q, const void* k, const void* v, void* o, float* ls
   if (int st = check_device(&dev)) return st;
   const int BH = B * H;
   int S = 1, tps = 1;
-  resolve_splits(BH, Nq, Nk, d, causal ? 1 : 0, splits, &S, &tps);
+  resolve_splits(BH, Nq, Nk, d, sizeof(T), causal ? 1 : 0, splits, &S, &tps);
   const size_t need = kvsplit_ws_bytes(BH, Nq, d, S);
   if (need > 0 && (!workspace || workspace_bytes_given < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)))
     return ATTN_ERR_INVALID;
@@ -421,8 +446,9 @@ int kvsplit_impl(const void* q, const void* k, const void* v, void* o, float* ls
   p.N = Nq;
   p.Nk = Nk;
   p.q_off = Nk - Nq;
+  const bool lean = use_lean(Nq, d, sizeof(T));
   p.BH = BH;
-  p.nblocks = (Nq + fwd_rows(d) - 1) / fwd_rows(d);
+  p.nblocks = lean ? 1 : (Nq + fwd_rows(d) - 1) / fwd_rows(d);
   p.splits = S;
   p.tps = tps;
   if (S > 1) {
@@ -436,7 +462,7 @@ int kvsplit_impl(const void* q, const void* k, const void* v, void* o, float* ls
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o_mul = 1.0f;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (int st = launch_fwd<T>(p, d, dev, s)) return st;
+  if (int st = lean ? launch_fwd_lean<T>(p, d, s) : launch_fwd<T>(p, d, dev, s)) return st;
   if (S == 1) return ATTN_OK;
   const long long rows = static_cast<long long>(BH) * Nq;
   const unsigned blocks = static_cast<unsigned>((rows + 7) / 8);
@@ -597,14 +623,14 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
 size_t attn_fwd_kvsplit_workspace_bytes(int B, int H, int Nq, int Nk, int d, int causal, int splits) {
   if (check_kvsplit_sizes(B, H, Nq, Nk, d, causal, splits) != 0) return 0;
   int S = 1, tps = 1;
-  resolve_splits(B * H, Nq, Nk, d, causal ? 1 : 0, splits, &S, &tps);
+  resolve_splits(B * H, Nq, Nk, d, 2, causal ? 1 : 0, splits, &S, &tps);
   return kvsplit_ws_bytes(B * H, Nq, d, S);
 }
 
 int attn_fwd_kvsplit_count(int B, int H, int Nq, int Nk, int d, int causal, int splits) {
   if (check_kvsplit_sizes(B, H, Nq, Nk, d, causal, splits) != 0) return 0;
   int S = 1, tps = 1;
-  resolve_splits(B * H, Nq, Nk, d, causal ? 1 : 0, splits, &S, &tps);
+  resolve_splits(B * H, Nq, Nk, d, 2, causal ? 1 : 0, splits, &S, &tps);
   return S;
 }
 

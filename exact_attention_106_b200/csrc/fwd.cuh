@@ -59,18 +59,25 @@ constexpr int kEmuPairs = 3;
 
 // T: the input element type (16-bit, or e4m3).  A tile row holds D
 // elements; tiles are stored as 128-byte swizzled chunks of 128 rows.
-template <int D, typename T>
+// kLean: a CTA of one 128-row sub-tile with a 2-slot K/V ring and 256 TMEM
+// columns, small enough that two CTAs share an SM.  For few query rows
+// (decode), where a second sub-tile would have no rows to work on, two such
+// CTAs keep the tensor core and the softmax of an SM overlapping.
+template <int D, typename T, bool kLean = false>
 struct FwdCfg {
   // 128-row query sub-tiles per CTA: two, except at head_dim 256, where one
   // sub-tile's S (128 columns) and O (256) already take 384 of the 512 TMEM
-  // columns.
-  static constexpr int kSub = (D == 256) ? 1 : 2;
+  // columns, and in the lean configuration.
+  static constexpr int kSub = (D == 256 || kLean) ? 1 : 2;
+  static_assert(!kLean || (D <= 128 && sizeof(T) == 2), "lean CTAs: 16-bit inputs, head_dim <= 128");
+  static constexpr uint32_t kTmemCols = kLean ? 256u : 512u;
+  static constexpr int kCtasPerSm = kLean ? 2 : 1;
   static constexpr int kRows = 128 * kSub;                     // query rows per CTA
   static constexpr int kThreads = 128 * kSub + 64;             // softmax warps, producer warp, MMA warp
   static constexpr uint32_t kElem = sizeof(T);
   static constexpr uint32_t kTile = 128u * D * kElem;          // one 128-row tile
   // K/V ring slots within the 227 KB of shared memory
-  static constexpr int kSlots = (kTile == 65536u) ? 2 : (kTile == 32768u) ? 4 : 8;
+  static constexpr int kSlots = kLean ? 2 : (kTile == 65536u) ? 2 : (kTile == 32768u) ? 4 : 8;
   static constexpr int kChunks = D * kElem / 128;              // 128-byte swizzle chunks per row
   static constexpr int kChunkElems = 128 / kElem;              // elements per chunk
   static constexpr int kKStep = 32 / kElem;                    // K of one MMA (32 bytes of a row)
@@ -83,9 +90,10 @@ struct FwdCfg {
 
 // T: the element type of Q, K and V (__nv_bfloat16, __half, or __nv_fp8_e4m3);
 // O has type Elem<T>::Out.
-template <int D, typename T>
-__global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, 1) attn_fwd_kernel(const __grid_constant__ FwdParams p) {
-  using C = FwdCfg<D, T>;
+template <int D, typename T, bool kLean = false>
+__global__ void __launch_bounds__(FwdCfg<D, T, kLean>::kThreads, FwdCfg<D, T, kLean>::kCtasPerSm)
+    attn_fwd_kernel(const __grid_constant__ FwdParams p) {
+  using C = FwdCfg<D, T, kLean>;
   using E = Elem<T>;
   using TO = typename E::Out;
   constexpr int kProducerWarp = 4 * C::kSub;
@@ -155,7 +163,7 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, 1) attn_fwd_kernel(con
     fence_barrier_init();
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(tmem_slot, 512);
+    tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -484,7 +492,7 @@ __global__ void __launch_bounds__(FwdCfg<D, T>::kThreads, 1) attn_fwd_kernel(con
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, C::kTmemCols);
 }
 
 }  // namespace exattn
