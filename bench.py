@@ -424,10 +424,37 @@ def run_sweep(args):
         rows.append(row)
         print(json.dumps(row), flush=True)
     for row in (kvsplit_points(dev, flush, burst, peak_src, args, only) + fp8_points(dev, flush, burst, args, only)
-                + hdim256_points(dev, flush, burst, args, only)):
+                + hdim256_points(dev, flush, burst, args, only) + fp16_points(dev, flush, burst, args, only)):
         rows.append(row)
         print(json.dumps(row), flush=True)
     return rows
+
+
+def fp16_points(dev, flush, burst, args, only):
+    """The long-context workload on fp16 tensors (attn_fwd_fp16 / attn_bwd_fp16),
+    forward and whole backward."""
+    import exact_attention_106_b200 as ex
+    from exact_attention_106_b200 import workloads as W
+    w = W.LONG_CONTEXT
+    name = w.name + "_fp16"
+    if only and name not in only:
+        return []
+    q, k, v, do = (x.to(dev) for x in W.make_inputs(w, dtype=torch.float16))
+    o = torch.empty_like(q)
+    lse = torch.empty(w.shape[:3], dtype=torch.float32, device=dev)
+    grads = tuple(torch.empty_like(q) for _ in range(3))
+    ws = ex.alloc_workspace(*w.shape, dev)
+    fwd = lambda: ex.forward(q, k, v, causal=True, scale=w.softmax_scale, out=o, lse=lse)  # noqa: E731
+    fwd()
+    bwd = lambda: ex.backward(q, k, v, o, lse, do, causal=True, scale=w.softmax_scale, workspace=ws,  # noqa: E731
+                              out=grads)
+    f_med, _, reps, clk = time_fn(fwd, dev, flush, args.sweep_reps, args.sweep_seconds)
+    b_med, _, _, _ = time_fn(bwd, dev, flush, args.sweep_reps, args.sweep_seconds)
+    ftf = w.fwd_flops() / (f_med * 1e-3) / 1e12
+    btf = w.bwd_flops() / (b_med * 1e-3) / 1e12
+    return [{"point": name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": True, "reps": reps,
+             "fwd_ms": f_med, "fwd_tflops": ftf, "bwd_ms_all_stages": b_med, "bwd_tflops_all_stages": btf,
+             "fwd_of_burst": ftf / burst, "bwd_of_burst": btf / burst, "clocks": clk}]
 
 
 def hdim256_points(dev, flush, burst, args, only):

@@ -65,3 +65,28 @@ def test_check_flag_raises_on_timeout(cuda_device):
         lib.attn_set_wait_timeout_ns(0)
     assert e1.value.status == _lib.ATTN_ERR_TIMEOUT and e2.value.status == _lib.ATTN_ERR_TIMEOUT
     assert ex.device_status() == 0
+
+
+def test_check_flag_raises_on_timeout_in_the_split_and_e4m3_forwards(cuda_device):
+    """The split-key and e4m3 forwards run the same kernel with the same
+    bounded waits: an injected stall surfaces as ATTN_ERR_TIMEOUT through
+    check=True, and the context stays usable."""
+    lib = _lib.load()
+    g = torch.Generator().manual_seed(9)
+    q = torch.randn((1, 2, 16, 128), generator=g).bfloat16().to(cuda_device)
+    kv = torch.randn((1, 2, 3000, 128), generator=g).bfloat16().to(cuda_device)
+    x8 = torch.randn((1, 2, 300, 128), generator=g).to(torch.float8_e4m3fn).to(cuda_device)
+    lib.attn_set_wait_timeout_ns(20_000_000)
+    lib.attn_debug_inject_stall(1)
+    try:
+        with pytest.raises(ex.ExattnError) as e1:
+            ex.forward_kvsplit(q, kv, kv, causal=True, splits=3, check=True)
+        with pytest.raises(ex.ExattnError) as e2:
+            ex.forward_fp8(x8, x8, x8, 1.0, 1.0, 1.0, causal=True, check=True)
+    finally:
+        lib.attn_debug_inject_stall(0)
+        lib.attn_set_wait_timeout_ns(0)
+    assert e1.value.status == _lib.ATTN_ERR_TIMEOUT and e2.value.status == _lib.ATTN_ERR_TIMEOUT
+    assert ex.device_status() == 0
+    o, _ = ex.forward_kvsplit(q, kv, kv, causal=True, splits=3, check=True)  # clean run afterwards
+    assert torch.isfinite(o.float()).all()
