@@ -272,6 +272,14 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o_mul = 1.0f;
+  // Short rows: each CTA does few key tiles, so its fixed costs (Q load,
+  // pipeline fill, epilogue) weigh; two lean CTAs per SM overlap them.
+  // Measured on the sweep: +3% to +18% up to N = 1024, 3-7% slower from 2048.
+  constexpr int kLeanMaxN = 1024;
+  if (N <= kLeanMaxN && use_lean(1, d, sizeof(T))) {
+    p.nblocks = (N + 127) / 128;
+    return launch_fwd_lean<T>(p, d, reinterpret_cast<cudaStream_t>(stream));
+  }
   return launch_fwd<T>(p, d, dev, reinterpret_cast<cudaStream_t>(stream));
 }
 
