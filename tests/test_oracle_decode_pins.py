@@ -136,6 +136,7 @@ def _dec_no_scale(q, k, v, scale, causal):
     return oracle.decode_head(q, k, v, 1.0, causal)
 
 
+@pytest.mark.filterwarnings("ignore::RuntimeWarning")  # a planted mask can hide every key of a row
 @pytest.mark.parametrize("bad", [_dec_top_left, _dec_off_by_one, _dec_no_scale], ids=lambda f: f.__name__)
 def test_planted_decode_mistakes_fail_a_pin(bad):
     failed = 0
