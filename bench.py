@@ -57,9 +57,10 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic():
+def recorded_traffic(workload):
     """Per-launch DRAM bytes of the backward main kernel from the committed ncu
-    summary, or None if absent or taken on a different kernel source."""
+    summary, or None if absent, taken on another workload or on a different
+    kernel source."""
     try:
         kv = {}
         with open(TRAFFIC_FILE) as f:
@@ -67,7 +68,7 @@ def recorded_traffic():
                 if ":" in line and not line.lstrip().startswith("#"):
                     a, b = line.split(":", 1)
                     kv[a.strip()] = b.strip()
-        if kv.get("kernel_source_sha256_16") != kernel_source_hash():
+        if kv.get("kernel_source_sha256_16") != kernel_source_hash() or kv.get("workload") != workload:
             return None
         return float(kv["traffic_bytes_per_launch"])
     except (OSError, KeyError, ValueError):
@@ -305,13 +306,15 @@ def run_ours(args, rank, world, local_rank):
                "sample": f"fp64 numpy oracle, fwd+bwd of heads 0..{nh - 1} of batch 0 of {w.name} "
                          f"(full length {N}); algorithmic flops of those heads / time"}
     spec_peak = 2250.0
+    tensor_mib = B * H * N * d * 2 / 2**20
     result = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d, "causal": w.causal,
                    "step": "forward + backward (all stages)", "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (Q, K, V, dO 128 MiB each per step)"},
+                   "l2": (f"inputs larger than L2 (Q, K, V, dO {tensor_mib:.0f} MiB each per step)"
+                          if 4 * tensor_mib > 126 else "inputs smaller than L2 (not flushed)")},
         "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
         "pct_of_peak": {"fwd_of_burst": fwd_tf / peak, "bwd_of_burst": bwd_tf / peak,
                         "fwd_of_sustained": fwd_tf / peak_sus, "bwd_of_sustained": bwd_tf / peak_sus,
@@ -322,7 +325,7 @@ def run_ours(args, rank, world, local_rank):
                      "bound": "tensor", "achieved": dom_tf, "peak": peak, "unit": "TFLOP/s",
                      "frac": dom_tf / peak, "peak_kind": f"bf16 burst ({peak_src})",
                      "frac_of_sustained": dom_tf / peak_sus,
-                     "traffic": recorded_traffic() if dominant == "bwd_dkdv" else None},
+                     "traffic": recorded_traffic(w.name) if dominant == "bwd_dkdv" else None},
         "cpu_baseline": cpu,
         "e2e": {"value": job_throughput(world, flops_step, e2e_steps, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
