@@ -33,16 +33,21 @@ std::atomic<unsigned int> g_debug_flags{0};                        // see attn_d
 // ------------------------------------------------------------------ checks
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// The kernels address rows of the [B*H, N padded to 128] views (the backward's
+// accumulator, TMA row coordinates) with 32-bit ints, and the grids count
+// 128-row tiles: both must stay below 2^31.  (A problem near the limit would
+// need over 256 GB per tensor, more than the device holds.)
+bool rows_fit(long long bh, int N) {
+  const long long rows = (static_cast<long long>(N) + 127) / 128 * 128;
+  return bh <= 0x7fffffffLL && rows * bh <= 0x7fffffffLL;
+}
+
 // 0 = proceed, 1 = empty problem (nothing to do), -1 = invalid
 int check_sizes(int B, int H, int N, int d) {
   if (B < 0 || H < 0 || N < 0) return -1;
   if (d != 64 && d != 128) return -1;
   if (B == 0 || H == 0 || N == 0) return 1;
-  const long long bh = static_cast<long long>(B) * H;
-  if (bh > 0x7fffffffLL) return -1;
-  const long long nblk = (static_cast<long long>(N) + 255) / 256;
-  if (nblk * bh > 0x7fffffffLL) return -1;  // grid size
-  return 0;
+  return rows_fit(static_cast<long long>(B) * H, N) ? 0 : -1;
 }
 
 bool check_scale(float scale) { return std::isfinite(scale) && scale > 0.f; }
@@ -55,10 +60,7 @@ int check_sizes_fwd(int B, int H, int N, int d) {
   if (d == 256) {
     if (B < 0 || H < 0 || N < 0) return -1;
     if (B == 0 || H == 0 || N == 0) return 1;
-    const long long bh = static_cast<long long>(B) * H;
-    if (bh > 0x7fffffffLL) return -1;
-    if ((static_cast<long long>(N) + 127) / 128 * bh > 0x7fffffffLL) return -1;
-    return 0;
+    return rows_fit(static_cast<long long>(B) * H, N) ? 0 : -1;
   }
   return check_sizes(B, H, N, d);
 }

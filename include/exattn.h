@@ -66,7 +66,8 @@ typedef enum attn_status {
   ATTN_OK = 0,
   ATTN_ERR_INVALID = 1,            /* bad argument: null/misaligned pointer, negative size,
                                       d not supported by the call, scale not finite or <= 0,
-                                      workspace too small, size overflow */
+                                      workspace too small, size overflow (B*H times N
+                                      rounded up to 128 must stay below 2^31) */
   ATTN_ERR_UNSUPPORTED_DEVICE = 2, /* current device is not sm_100 (B200) */
   ATTN_ERR_LAUNCH = 3,             /* a CUDA call failed (launch, attribute, tensor map) */
   ATTN_ERR_TIMEOUT = 4             /* a device-side wait ran out (see above) */

@@ -54,6 +54,9 @@ def fwd(lib, **kw):
     dict(d=96), dict(d=32), dict(d=512), dict(B=-1), dict(N=-5), dict(scale=0.0), dict(scale=-1.0),
     dict(scale=float("inf")), dict(scale=float("nan")), dict(q=None), dict(lse=None),
     dict(k=P + 8), dict(o=P + 2),
+    # padded rows of the [B*H, N] view past 2^31 - 1 (the kernels' 32-bit row coordinates)
+    dict(H=1 << 16, N=1 << 16), dict(H=1 << 14, N=1 << 17), dict(B=1 << 15, H=1 << 16, N=1),
+    dict(H=1 << 16, N=1 << 16, d=256), dict(H=1 << 14, N=(1 << 17) - 127, d=128),
 ])
 def test_fwd_rejects_bad_arguments_on_host(lib, kw):
     assert fwd(lib, **kw) == _lib.ATTN_ERR_INVALID
