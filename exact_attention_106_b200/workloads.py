@@ -16,6 +16,11 @@ Recipe (shared by tests and the benchmark):
     "Flash Attention: From Theory to Implementation", introduction;
   * the "stability" workload multiplies Q by 8 on heads [H/2, H) of every
     batch, in float32 before the bf16 cast (x8 is exact in bf16).
+  * a problem too large to draw whole on the host (the 64-bit offsets case)
+    is drawn one head at a time for the heads that are checked
+    (``make_head``: seed = base + 10 x (b x H + h) + tensor index); the
+    other heads are filler of the same distribution, which cannot reach a
+    checked head (every head is an independent problem).
 """
 from __future__ import annotations
 
@@ -84,6 +89,12 @@ def make_inputs(w: Workload, with_grad_out: bool = True, dtype: torch.dtype = to
     return tuple(out)
 
 
+def make_head(w: Workload, b: int, h: int, dtype: torch.dtype = torch.bfloat16):
+    """(q, k, v, do) of head (b, h) alone, each [N, d], on the host."""
+    base = w.seed_base + 10 * (b * w.H + h)
+    return tuple(_seeded_normal((w.N, w.d), base + t).to(dtype) for t in range(4))
+
+
 # ---------------------------------------------------------------------------
 # The named workloads.  Sizes follow the shapes the pages use: head_dim 64/128,
 # 32 heads, sequence lengths from 512 to 32768.
@@ -95,6 +106,12 @@ LLAMA_BLOCK = Workload("llama_block_4x16x4096x128_causal", 4, 16, 4096, 128, Tru
 LONG_CONTEXT = Workload("long_context_1x32x16384x128_causal", 1, 32, 16384, 128, True, 4000)
 
 NAMED = [TINY, SMALL_CAUSAL_STABILITY, LLAMA_BLOCK, LONG_CONTEXT]
+
+# Element offsets past 2^31: the last head of each [B, H, N, d] tensor starts
+# at element (H - 1) * N * d = 2.19e9, and its rows of the padded backward
+# accumulator past 2^31 elements too; N is ragged (64 full tiles + 37 rows).
+# 4.4 GB per bf16 tensor, about 45 GB on the device for forward + backward.
+LARGE_OFFSETS = Workload("offsets64_1x2080x8229x128_causal", 1, 2080, 8229, 128, True, 5000)
 
 SWEEP_TOKENS = 16384
 SWEEP_N = [512, 1024, 2048, 4096, 8192, 16384]
