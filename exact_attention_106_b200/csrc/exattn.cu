@@ -347,16 +347,23 @@ int block_tiles(int qb, int rows, int Nq, int Nk, int causal) {
 // then 1.  Otherwise each candidate S is simulated: the CTAs, in launch order
 // (heaviest query block first), are handed to the SMs as they free up, a CTA
 // costing its key tiles plus a fixed start-up cost, and S > 1 pays for the
-// merge pass; the S with the shortest makespan wins.  The result depends only
-// on the sizes and the SM count and is cached.
+// merge pass; the S with the shortest makespan wins.  The choice is made on
+// whole tiles (Nq and Nk rounded up to the query block and the key tile), so
+// that the calls of a decode loop, whose key count grows by one per step,
+// share one plan per 128 keys; it depends only on those counts and the SM
+// count and is cached (at most kMaxPlans entries; the cache starts over
+// when full).
+constexpr size_t kMaxPlans = 4096;
 int choose_splits(int BH, int Nq, int Nk, int causal, int rows, int per_sm) {
   const int sms = sm_count() * per_sm;  // CTAs resident at once
   const int nblocks = (Nq + rows - 1) / rows;
   const int ntk = (Nk + 127) / 128;
   if (static_cast<long long>(BH) * nblocks >= 4LL * sms || ntk == 1) return 1;
+  Nq = nblocks * rows;
+  Nk = ntk * 128;
   static std::mutex mu;
   static std::map<std::tuple<int, int, int, int, int, int>, int> cache;
-  const auto key = std::make_tuple(BH, Nq, Nk, causal, sms, rows);  // sms counts resident CTAs
+  const auto key = std::make_tuple(BH, nblocks, ntk, causal, sms, rows);  // sms counts resident CTAs
   {
     std::lock_guard<std::mutex> lock(mu);
     auto it = cache.find(key);
@@ -391,6 +398,7 @@ int choose_splits(int BH, int Nq, int Nk, int causal, int rows, int per_sm) {
     }
   }
   std::lock_guard<std::mutex> lock(mu);
+  if (cache.size() >= kMaxPlans) cache.clear();
   cache[key] = best;
   return best;
 }

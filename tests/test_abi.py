@@ -147,3 +147,14 @@ def test_kvsplit_plan_on_host(lib):
     assert lib.attn_fwd_kvsplit_count(1, 1, 1000, 1000, 64, 0, 4) == 4
     # 5 asked over 8 key tiles: ranges of ceil(8 / 5) = 2 tiles, so 4 of them
     assert lib.attn_fwd_kvsplit_count(1, 1, 1000, 1000, 64, 0, 5) == 4
+
+
+def test_kvsplit_plan_is_per_whole_tile(lib):
+    """A decode loop's key count grows by one per step: the automatic plan is
+    made on whole key tiles, so the counts within one 128-key tile share it
+    (and the planner's cache holds one entry per tile, not per step)."""
+    for B, H, Nq in ((8, 32, 1), (8, 32, 16), (1, 8, 16)):
+        for t0 in (256, 781):
+            plans = {lib.attn_fwd_kvsplit_count(B, H, Nq, nk, 128, 1, 0) for nk in range(128 * t0 + 1, 128 * (t0 + 1) + 1)}
+            assert len(plans) == 1, (B, H, Nq, t0, plans)
+            assert 1 <= plans.pop() <= 64
