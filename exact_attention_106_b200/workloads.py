@@ -107,6 +107,10 @@ LONG_CONTEXT = Workload("long_context_1x32x16384x128_causal", 1, 32, 16384, 128,
 
 NAMED = [TINY, SMALL_CAUSAL_STABILITY, LLAMA_BLOCK, LONG_CONTEXT]
 
+# A second small case, past the short-row (N <= 1024) forward configuration:
+# the two-sub-tile forward and the head_dim-128 backward, ragged last tile.
+SMOKE_D128 = Workload("smoke_1x2x1280x128_causal", 1, 2, 1280, 128, True, 6000)
+
 # Element offsets past 2^31: the last head of each [B, H, N, d] tensor starts
 # at element (H - 1) * N * d = 2.19e9, and its rows of the padded backward
 # accumulator past 2^31 elements too; N is ragged (64 full tiles + 37 rows).
