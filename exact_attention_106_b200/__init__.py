@@ -33,6 +33,7 @@ def _stream(device: torch.device) -> int:
 
 # element type -> (forward, backward) entry points of the C ABI
 _ENTRY = {torch.bfloat16: ("attn_fwd", "attn_bwd"), torch.float16: ("attn_fwd_fp16", "attn_bwd_fp16")}
+_KVSPLIT_ENTRY = {torch.bfloat16: "attn_fwd_kvsplit", torch.float16: "attn_fwd_kvsplit_fp16"}
 
 
 def _check_qkv(*ts: torch.Tensor) -> None:
@@ -111,13 +112,15 @@ def forward_kvsplit(q, k, v, causal: bool = False, scale: Optional[float] = None
     """Forward over Nq queries and Nk keys with the keys split into ranges
     (attn_fwd_kvsplit): decode (Nq small, Nk long) and long rows.
 
-    q: [B, H, Nq, d], k, v: [B, H, Nk, d], CUDA bfloat16, contiguous.  Under
-    ``causal`` the queries are the last Nq positions (query i sees keys
-    j <= Nk - Nq + i).  ``splits`` 0 lets the library choose.
+    q: [B, H, Nq, d], k, v: [B, H, Nk, d], CUDA bfloat16 or float16 (all
+    three alike), contiguous.  Under ``causal`` the queries are the last Nq
+    positions (query i sees keys j <= Nk - Nq + i).  ``splits`` 0 lets the
+    library choose.
     """
     for t in (q, k, v):
-        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous() and t.dim() == 4):
-            raise ValueError("expected contiguous CUDA bfloat16 tensors [B, H, N, d]")
+        if not (t.is_cuda and t.dtype in _KVSPLIT_ENTRY and t.dtype == q.dtype and t.is_contiguous()
+                and t.dim() == 4):
+            raise ValueError("expected contiguous CUDA bfloat16 or float16 tensors [B, H, N, d] of one dtype")
     B, H, Nq, d = q.shape
     if k.shape != (B, H, k.shape[2], d) or v.shape != k.shape:
         raise ValueError("k and v must be [B, H, Nk, d] with q's B, H, d")
@@ -128,11 +131,12 @@ def forward_kvsplit(q, k, v, causal: bool = False, scale: Optional[float] = None
     ws = workspace
     if ws is None:
         ws = torch.empty(max(1, need), dtype=torch.uint8, device=q.device)
-    _lib.check("attn_fwd_kvsplit", _lib.load().attn_fwd_kvsplit(
+    name = _KVSPLIT_ENTRY[q.dtype]
+    _lib.check(name, getattr(_lib.load(), name)(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse_t.data_ptr(), B, H, Nq, Nk, d,
         _scale(d, scale), int(causal), int(splits), ws.data_ptr(), ws.numel(), _stream(q.device)))
     if check:
-        _check_status("attn_fwd_kvsplit", q.device)
+        _check_status(name, q.device)
     return o, lse_t
 
 

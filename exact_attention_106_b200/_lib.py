@@ -28,6 +28,7 @@ SIGNATURES = {
     "attn_bwd_dq_convert": (_i, [_vp, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
     "attn_fwd_fp8": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _f, _f, _f, _vp]),
     "attn_fwd_kvsplit": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _i, _vp, _sz, _vp]),
+    "attn_fwd_kvsplit_fp16": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _i, _vp, _sz, _vp]),
     "attn_fwd_kvsplit_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "attn_fwd_kvsplit_count": (_i, [_i, _i, _i, _i, _i, _i, _i]),
     "attn_fwd_fp16": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp]),

@@ -659,6 +659,13 @@ int attn_fwd_kvsplit(const void* q, const void* k, const void* v, void* o, float
                                      workspace_bytes_given, stream);
 }
 
+int attn_fwd_kvsplit_fp16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
+                          int Nk, int d, float scale, int causal, int splits, void* workspace,
+                          size_t workspace_bytes_given, attn_stream_t stream) {
+  return kvsplit_impl<__half>(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, splits, workspace,
+                              workspace_bytes_given, stream);
+}
+
 // ------------------------------------------------------------- e4m3 forward
 int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
                  float scale, int causal, float q_descale, float k_descale, float v_descale, attn_stream_t stream) {

@@ -155,6 +155,7 @@ int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* ls
  * machine under-filled.
  *
  *   q, o  : bf16 [B,H,Nq,d] (in / out)     k, v : bf16 [B,H,Nk,d] (in)
+ *           (fp16 through attn_fwd_kvsplit_fp16, below)
  *   lse   : fp32 [B,H,Nq] (out), natural-log logsumexp of each scaled score row
  *   causal: the Nq queries are the LAST Nq positions of the Nk-token
  *           sequence: query i sees key j iff j <= Nk - Nq + i (for Nq = Nk
@@ -208,6 +209,13 @@ int attn_fwd_fp16(const void* q, const void* k, const void* v, void* o, float* l
 int attn_bwd_fp16(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                   void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
                   void* workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/* attn_fwd_kvsplit() on fp16 q, k, v and o; attn_fwd_kvsplit_workspace_bytes()
+ * and attn_fwd_kvsplit_count() apply unchanged (they do not depend on which
+ * 16-bit type is used). */
+int attn_fwd_kvsplit_fp16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
+                          int Nk, int d, float scale, int causal, int splits, void* workspace,
+                          size_t workspace_bytes, attn_stream_t stream);
 
 /*
  * Backward without any device allocation: attn_bwd() run on scratch memory

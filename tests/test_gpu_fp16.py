@@ -71,3 +71,14 @@ def test_fp16_and_bf16_paths_are_different_kernels(cuda_device):
         ref = oracle_ref(*(t.double() for t in x), True, 0.1)  # exact fp32 inputs
         errs[dt] = float(np.max(np.abs(got["o"] - ref["o"])))
     assert errs[F16] < errs[torch.bfloat16], errs
+
+
+def test_fp16_long_context_sampled_heads(cuda_device):
+    """1x32x16384x128 causal in fp16, the shape of the fp16 bench point: the
+    full launch, the first and last heads against the oracle."""
+    w = W.LONG_CONTEXT
+    q, k, v, do = W.make_inputs(w, dtype=F16)
+    got = run_cuda(q, k, v, do, w.causal, w.softmax_scale)
+    heads = [(0, 0), (0, 31)]
+    ref = oracle_ref(q, k, v, do, w.causal, w.softmax_scale, heads=heads)
+    check_all(got, ref, heads=heads, what="fp16 " + w.name)

@@ -75,6 +75,28 @@ def test_fp8_llama_block_shape_sampled_heads(cuda_device):
         check_lse(lse[b, h], lse_ref[b, h], f"fp8 head {b},{h}")
 
 
+def test_fp8_long_context_sampled_heads(cuda_device):
+    """1x32x16384x128 causal, the shape and inputs of the e4m3 bench point (the
+    long-context draws, quantized per tensor): the full launch, the first and
+    last heads against the oracle."""
+    w = W.LONG_CONTEXT
+    x = W.make_inputs(w, with_grad_out=False, dtype=torch.float32)[:3]
+    (q8, qs, qr), (k8, ks, kr), (v8, vs, vr) = (_quantize(t) for t in x)
+    o, lse = ex.forward_fp8(q8.to(cuda_device), k8.to(cuda_device), v8.to(cuda_device), qs, ks, vs, causal=True)
+    torch.cuda.synchronize()
+    assert ex.device_status() == 0
+    heads = [(0, 0), (0, 31)]
+    o = np.stack([to_np(o[b, h]) for b, h in heads])
+    lse = np.stack([to_np(lse[b, h]) for b, h in heads])
+    o_ref, lse_ref = oracle.forward(qr, kr, vr, w.softmax_scale, True, heads=heads)
+    o_abs, _ = oracle.forward(qr, kr, vr.abs(), w.softmax_scale, True, heads=heads)
+    for i, (b, h) in enumerate(heads):
+        bound = 2.0 ** -4 * o_abs[b, h] + 2.0 ** -8 * np.abs(o_ref[b, h]) + 1e-3
+        excess = float(np.max(np.abs(o[i] - o_ref[b, h]) - bound))
+        assert excess <= 0, f"fp8 long context head {b},{h}: O error exceeds its bound by {excess:.3e}"
+        check_lse(lse[i], lse_ref[b, h], f"fp8 long context head {b},{h}")
+
+
 def test_fp8_large_scores_stability(cuda_device):
     """Q x 8: near one-hot rows, where the reference maximum moves often."""
     g = torch.Generator().manual_seed(5)

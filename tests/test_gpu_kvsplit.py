@@ -45,6 +45,32 @@ def test_decode_shapes(cuda_device, nq, nk, d, causal, splits):
     check_lse(lse, lse_ref, what)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("nq,nk,d,splits", [(1, 4097, 128, 0), (16, 4097, 64, 3), (130, 1000, 128, 0),
+                                            (7, 300, 64, 1), (1, 20000, 128, 0)])
+def test_decode_shapes_fp16(cuda_device, nq, nk, d, causal, splits):
+    """attn_fwd_kvsplit_fp16: the same shapes on fp16 inputs (the oracle takes
+    the fp16 values upcast exactly)."""
+    B, H = 2, 3
+    g = torch.Generator().manual_seed(nq * 17 + nk + d)
+    q, k, v = (torch.randn(shape, generator=g).half() for shape in ((B, H, nq, d), (B, H, nk, d), (B, H, nk, d)))
+    scale = 1 / math.sqrt(d)
+    o, lse = _run(q, k, v, causal, scale, splits, cuda_device)
+    o_ref, lse_ref = oracle.decode(q, k, v, scale, causal)
+    what = f"fp16 nq={nq} nk={nk} d={d} causal={causal} splits={splits}"
+    check_o(o, o_ref, what)
+    check_lse(lse, lse_ref, what)
+
+
+def test_kvsplit_rejects_mixed_dtypes(cuda_device):
+    q = torch.zeros((1, 1, 1, 64), dtype=torch.float16, device=cuda_device)
+    k = torch.zeros((1, 1, 8, 64), dtype=torch.bfloat16, device=cuda_device)
+    with pytest.raises(ValueError):
+        ex.forward_kvsplit(q, k, k)
+    with pytest.raises(ValueError):
+        ex.forward_kvsplit(q.float(), k.float(), k.float())
+
+
 @pytest.mark.parametrize("N,splits", [(1000, 3), (257, 2), (2048, 16), (640, 64)])
 def test_square_problem_with_forced_splits(cuda_device, N, splits):
     """Nq = Nk: the causal mask is the square one of attn_fwd; splitting the
