@@ -121,10 +121,12 @@ def test_host_call_rejects_bad_arguments(lib):
 def test_kvsplit_and_fp8_reject_bad_arguments_on_host(lib):
     v = _lib.ATTN_ERR_INVALID
     # causal with more queries than keys; no keys; negative split count; d = 96
-    assert lib.attn_fwd_kvsplit(P, P, P, P, P, 1, 1, 20, 10, 64, 0.1, 1, 0, P, 1 << 20, None) == v
-    assert lib.attn_fwd_kvsplit(P, P, P, P, P, 1, 1, 20, 0, 64, 0.1, 0, 0, P, 1 << 20, None) == v
-    assert lib.attn_fwd_kvsplit(P, P, P, P, P, 1, 1, 20, 20, 64, 0.1, 0, -1, P, 1 << 20, None) == v
-    assert lib.attn_fwd_kvsplit(P, P, P, P, P, 1, 1, 20, 20, 96, 0.1, 0, 0, P, 1 << 20, None) == v
+    for fn in (lib.attn_fwd_kvsplit, lib.attn_fwd_kvsplit_fp16):
+        assert fn(P, P, P, P, P, 1, 1, 20, 10, 64, 0.1, 1, 0, P, 1 << 20, None) == v
+        assert fn(P, P, P, P, P, 1, 1, 20, 0, 64, 0.1, 0, 0, P, 1 << 20, None) == v
+        assert fn(P, P, P, P, P, 1, 1, 20, 20, 64, 0.1, 0, -1, P, 1 << 20, None) == v
+        assert fn(P, P, P, P, P, 1, 1, 20, 20, 96, 0.1, 0, 0, P, 1 << 20, None) == v
+        assert fn(None, None, None, None, None, 1, 1, 0, 10, 64, 0.1, 0, 0, None, 0, None) == 0
     assert lib.attn_fwd_kvsplit_count(1, 1, 20, 10, 64, 1, 0) == 0
     # e4m3: d must be 128, descale factors finite and > 0
     assert lib.attn_fwd_fp8(P, P, P, P, P, 1, 1, 8, 64, 0.1, 0, 1.0, 1.0, 1.0, None) == v
