@@ -45,6 +45,7 @@ struct BwdParams {
   int ntiles;  // ceil(N / 128)
   int head_group;  // heads whose CTAs are scheduled together (L2 reuse of Q/dO/dQ)
   int causal;
+  int paired;      // causal items taken in pairs (j, ntiles - 1 - j); see the kernel
   float scale;
   float scale_log2;
   unsigned long long timeout_ns;
@@ -64,7 +65,7 @@ struct BwdCfg {
   // a whole 128-column dQ partial.  This fits if kRegsDrain - R <= R - kRegsSide,
   // i.e. R >= kRegsMin; the host refuses to launch a build with fewer.
   static constexpr int kRegsDrain = 168;
-  static constexpr int kRegsSide = 64;
+  static constexpr int kRegsSide = 80;
   static constexpr int kRegsMin = (kRegsDrain + kRegsSide + 1) / 2;
   static constexpr int kRegsMax = 65536 / kThreads;
   static_assert(kRegsMin <= kRegsMax, "register split cannot fit");
@@ -105,7 +106,10 @@ __device__ __forceinline__ void bwd_issue_t(uint32_t d_tmem, SmemDesc dKm, uint3
 }
 
 // T: the 16-bit element type of Q, K, V, dO and the gradients.
-template <int D, typename T>
+// kPersist: the CTA walks several work units (see below); otherwise it runs
+// the single unit blockIdx.x, and the step and item counters fold to their
+// first values at compile time.
+template <int D, typename T, bool kPersist>
 __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant__ BwdParams p) {
   using C = BwdCfg<D>;
   using E = Elem<T>;
@@ -144,19 +148,49 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
   // which only loads after that drain has released the stage, so the
   // barrier can never run two phases ahead of its waiter
   uint64_t* bar_dvdone = bars + 18;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
+  uint64_t* bar_accfree = bars + 20;  // dK, dV of an item read out by the epilogue (256 arrivals)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 21);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int N = p.N;
   const int ntq = p.ntiles;  // query tiles
-  // Key tile 0 first (under the causal mask it sees the most query tiles), a
-  // few heads at a time.
-  int j, bh;
-  grouped_order(static_cast<int>(blockIdx.x), p.ntiles, p.BH, p.head_group, j, bh);
-  const int i0 = p.causal ? j : 0;
-  const int n = ntq - i0;  // >= 1
+  // The CTA is persistent: it works through the items (key tile j, head bh)
+  // blockIdx.x, blockIdx.x + gridDim.x, ...  Item order: key tile 0 first
+  // (under the causal mask it sees the most query tiles), a few heads at a
+  // time.  Every role walks the same sequence; a step's rings and barriers
+  // take their phases from its index g in the CTA's whole sequence of steps,
+  // so that one item's loads and products start while the previous item's
+  // epilogue runs.
+  //
+  // The host either launches one CTA per item (each CTA then runs a single
+  // unit, and the hardware hands out the items as SMs free up), or, for
+  // short problems where a CTA's start-up and epilogue weigh, one CTA per SM
+  // with p.paired set under the causal mask.  Key tile j then sees ntq - j
+  // query tiles, so the items are taken in pairs (j, ntq - 1 - j) of one
+  // head, heavier first: every pair costs ntq + 1 steps, and a fixed stride
+  // over equal units balances the SMs as well as the hardware's scheduling
+  // would (with an odd ntq the middle tile stands alone, last in its head's
+  // order).  Otherwise every item is its own unit.
+  const int npt = (ntq + 1) / 2;
+  const bool paired = kPersist && p.causal && p.paired;
+  constexpr int kHalves = kPersist ? 2 : 1;
+  const int units = (paired ? npt : ntq) * p.BH;
+  auto unit_item = [&](int u, int half, int& j, int& bh, int& i0, int& n) -> bool {
+    int r;
+    grouped_order(u, paired ? npt : ntq, p.BH, p.head_group, r, bh);
+    if (!paired) {
+      j = r;
+      i0 = p.causal ? j : 0;
+      n = ntq - i0;  // >= 1
+      return half == 0;
+    }
+    j = half ? ntq - 1 - r : r;
+    i0 = j;
+    n = ntq - j;  // >= 1
+    return !(half && j == r);
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(bar_kv, 1);
@@ -177,6 +211,7 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
     mbar_init(bar_drain, 2);
     mbar_init(&bar_dvdone[0], 1);
     mbar_init(&bar_dvdone[1], 1);
+    mbar_init(bar_accfree, 256);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -199,38 +234,75 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       prefetch_tensormap(&p.tm_k);
       prefetch_tensormap(&p.tm_v);
       prefetch_tensormap(&p.tm_do);
-      const bool kv_issued = !(p.debug_flags & kDebugSkipFirstKV);  // else: injected stall
-      if (kv_issued) {
-        mbar_arrive_expect_tx(bar_kv, 2 * TILE);
-#pragma unroll
-        for (int c = 0; c < C::kChunks; ++c) {
-          tma_load_3d(sK + c * 16384, &p.tm_k, bar_kv, c * 64, j * 128, bh);
-          tma_load_3d(sV + c * 16384, &p.tm_v, bar_kv, c * 64, j * 128, bh);
-        }
-      }
       int lq[2] = {-1, -1}, ld[2] = {-1, -1};  // parity of the last loads into each stage
-      for (int it = 0; it < n; ++it) {
-        const int st = it & 1;
-        const uint32_t ph = (it >> 1) & 1;
-        const int i = i0 + it;
-        if (!mbar_wait(&bar_qempty[st], ph ^ 1u, abort_flag, tmo, 201)) break;
-        mbar_arrive_expect_tx(&bar_qfull[st], TILE + 1024);
+      int lkv = -1;                            // parity of the last K, V load
+      bool ok = true;
+      int g0_ = 0, t_ = 0;  // first step of the item, items done
+      for (int wu = blockIdx.x; wu < units && ok; wu += kPersist ? static_cast<int>(gridDim.x) : units)
+      for (int half = 0; half < kHalves && ok; ++half) {
+        int j, bh, i0, n;
+        if (!unit_item(wu, half, j, bh, i0, n)) continue;
+        const int g0 = kPersist ? g0_ : 0;  // this item's first step
+        const int t = kPersist ? t_ : 0;    // items before this one
+        auto load_kv = [&]() {
+          if (t > 0 || !(p.debug_flags & kDebugSkipFirstKV)) {  // else: injected stall
+            mbar_arrive_expect_tx(bar_kv, 2 * TILE);
 #pragma unroll
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(sQ + st * TILE + c * 16384, &p.tm_q, &bar_qfull[st], c * 64, i * 128, bh);
-        const size_t vrow = static_cast<size_t>(bh) * p.Np + static_cast<size_t>(i) * 128;
-        bulk_load(sVec + st * 256, p.lse2 + vrow, 512, &bar_qfull[st]);
-        bulk_load(sVec + st * 256 + 128, p.dvec + vrow, 512, &bar_qfull[st]);
-        if (st == 0) lq[0] = static_cast<int>(ph); else lq[1] = static_cast<int>(ph);
-        if (!mbar_wait(&bar_doempty[st], ph ^ 1u, abort_flag, tmo, 202)) break;
-        mbar_arrive_expect_tx(&bar_dofull[st], TILE);
+            for (int c = 0; c < C::kChunks; ++c) {
+              tma_load_3d(sK + c * 16384, &p.tm_k, bar_kv, c * 64, j * 128, bh);
+              tma_load_3d(sV + c * 16384, &p.tm_v, bar_kv, c * 64, j * 128, bh);
+            }
+            lkv = t & 1;
+          }
+        };
+        if (t == 0) load_kv();  // a fresh CTA: K and V first, the first S^T needs K at once
+        for (int it = 0; it < n; ++it) {
+          const int g = g0 + it;
+          const int st = g & 1;
+          const uint32_t ph = (g >> 1) & 1;
+          const int i = i0 + it;
+          if (!mbar_wait(&bar_qempty[st], ph ^ 1u, abort_flag, tmo, 201)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar_qfull[st], TILE + 1024);
 #pragma unroll
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(sDO + st * TILE + c * 16384, &p.tm_do, &bar_dofull[st], c * 64, i * 128, bh);
-        if (st == 0) ld[0] = static_cast<int>(ph); else ld[1] = static_cast<int>(ph);
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_3d(sQ + st * TILE + c * 16384, &p.tm_q, &bar_qfull[st], c * 64, i * 128, bh);
+          const size_t vrow = static_cast<size_t>(bh) * p.Np + static_cast<size_t>(i) * 128;
+          bulk_load(sVec + st * 256, p.lse2 + vrow, 512, &bar_qfull[st]);
+          bulk_load(sVec + st * 256 + 128, p.dvec + vrow, 512, &bar_qfull[st]);
+          if (st == 0) lq[0] = static_cast<int>(ph); else lq[1] = static_cast<int>(ph);
+          if (!mbar_wait(&bar_doempty[st], ph ^ 1u, abort_flag, tmo, 202)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar_dofull[st], TILE);
+#pragma unroll
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_3d(sDO + st * TILE + c * 16384, &p.tm_do, &bar_dofull[st], c * 64, i * 128, bh);
+          if (st == 0) ld[0] = static_cast<int>(ph); else ld[1] = static_cast<int>(ph);
+          if (it == 0 && t > 0) {
+            // A later item's K_j, V_j, after its first Q and dO, once every
+            // product of the previous item that reads K or V is done: S^T and
+            // dP^T (the last dP^T commit covers the S^T before it) and dQ of
+            // its last step g0 - 1.  dK and dV read neither, so the load
+            // overlaps them and the item's epilogue.  The two barriers cannot
+            // be a phase further on: this item's dP^T and dQ need the K and V
+            // loaded here.
+            if (!(mbar_wait(bar_dp, (g0 - 1) & 1, abort_flag, tmo, 206) &&
+                  mbar_wait(bar_dqfull, (g0 - 1) & 1, abort_flag, tmo, 227))) {
+              ok = false;
+              break;
+            }
+            load_kv();
+          }
+        }
+        g0_ += n;
+        ++t_;
       }
       // Let every copy issued so far land before the CTA can exit.
-      if (kv_issued) drain_wait(bar_kv, 0, 203);
+      if (lkv >= 0) drain_wait(bar_kv, static_cast<uint32_t>(lkv), 203);
       for (int s = 0; s < 2; ++s) {
         if (lq[s] >= 0) drain_wait(&bar_qfull[s], static_cast<uint32_t>(lq[s]), 204);
         if (ld[s] >= 0) drain_wait(&bar_dofull[s], static_cast<uint32_t>(ld[s]), 205);
@@ -253,74 +325,139 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       constexpr uint32_t oK = C::kOffK, oV = C::kOffV, oQ = C::kOffQ, oDO = C::kOffDO, oDS = C::kOffDS;
       if (warp == kMmaWarp) {
         // S^T = K Q_i^T, dP^T = V dO_i^T, dV += P^T dO_i
-        bool ok = mbar_wait(bar_kv, 0, abort_flag, tmo, 210) && mbar_wait(&bar_qfull[0], 0, abort_flag, tmo, 211) &&
-                  mbar_wait(&bar_dofull[0], 0, abort_flag, tmo, 212);
-        if (ok) {
+        bool ok = true;
+        int g0_ = 0, t_ = 0;
+        for (int wu = blockIdx.x; wu < units && ok; wu += kPersist ? static_cast<int>(gridDim.x) : units)
+        for (int half = 0; half < kHalves && ok; ++half) {
+          int j, bh, i0, n;
+          if (!unit_item(wu, half, j, bh, i0, n)) continue;
+          const int g0 = kPersist ? g0_ : 0;  // this item's first step
+          const int t = kPersist ? t_ : 0;    // items before this one
+          const int st0 = g0 & 1;
+          const uint32_t ph0 = (g0 >> 1) & 1;
+          ok = mbar_wait(bar_kv, t & 1, abort_flag, tmo, 210) && mbar_wait(&bar_qfull[st0], ph0, abort_flag, tmo, 211);
+          if (!ok) break;
           tc_fence_after();
-          bwd_issue_t<D, T>(tmem + C::kColS, dKm, oK, oQ);
+          bwd_issue_t<D, T>(tmem + C::kColS, dKm, oK, oQ + st0 * TILE);
           tc_commit(bar_s);
-          bwd_issue_t<D, T>(tmem + C::kColDP, dKm, oV, oDO);
-          tc_commit(bar_dp);
-        }
-        for (int it = 0; it < n && ok; ++it) {
-          const int st = it & 1;
-          const int st1 = (it + 1) & 1;
-          const uint32_t ph1 = ((it + 1) >> 1) & 1;
-          // dV += P^T dO_i   (A = P^T from TMEM, K = 128 queries; queries 0..63
-          // sit in columns [0,32) of the score block, 64..127 in [64,96))
-          if (!mbar_wait(bar_p, it & 1, abort_flag, tmo, 213)) break;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + C::kColDV, tmem + C::kColS + (kk >> 2) * 64 + (kk & 3) * 8,
-                   desc_at(dMN, oDO + st * TILE + kk * 2048), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
-          tc_commit(&bar_dvdone[st]);  // also dP_i: both readers of dO_i are done
-          if (it + 1 < n) {
-            // next S^T as early as possible: its softmax overlaps dQ, dK of tile it
-            if (!mbar_wait(&bar_qfull[st1], ph1, abort_flag, tmo, 214)) break;
-            tc_fence_after();
-            bwd_issue_t<D, T>(tmem + C::kColS, dKm, oK, oQ + st1 * TILE);
-            tc_commit(bar_s);
-            // dP^T(it+1) overwrites dP^T(it), read once dS_i is written, and at
-            // d = 128 also the dQ partial, free once the drain has read it
-            if (!mbar_wait(bar_ds, it & 1, abort_flag, tmo, 215)) break;
-            if (D == 128 && !mbar_wait(bar_dqfree, it & 1, abort_flag, tmo, 217)) break;
-            if (!mbar_wait(&bar_dofull[st1], ph1, abort_flag, tmo, 218)) break;
-            tc_fence_after();
-            bwd_issue_t<D, T>(tmem + C::kColDP, dKm, oV, oDO + st1 * TILE);
-            tc_commit(bar_dp);
+          // dP^T overwrites the previous step's dP^T, read once its dS is
+          // written, and at d = 128 also that step's dQ partial
+          if (g0 > 0) {
+            ok = mbar_wait(bar_ds, (g0 - 1) & 1, abort_flag, tmo, 207) &&
+                 (D != 128 || mbar_wait(bar_dqfree, (g0 - 1) & 1, abort_flag, tmo, 208));
+            if (!ok) break;
           }
+          ok = mbar_wait(&bar_dofull[st0], ph0, abort_flag, tmo, 212);
+          if (!ok) break;
+          tc_fence_after();
+          bwd_issue_t<D, T>(tmem + C::kColDP, dKm, oV, oDO + st0 * TILE);
+          tc_commit(bar_dp);
+          for (int it = 0; it < n; ++it) {
+            const int g = g0 + it;
+            const int st = g & 1;
+            const int st1 = (g + 1) & 1;
+            const uint32_t ph1 = ((g + 1) >> 1) & 1;
+            // dV += P^T dO_i   (A = P^T from TMEM, K = 128 queries; queries 0..63
+            // sit in columns [0,32) of the score block, 64..127 in [64,96)); the
+            // item's first dV starts over once the previous item's dV is read out
+            if (!mbar_wait(bar_p, g & 1, abort_flag, tmo, 213) ||
+                (it == 0 && t > 0 && !mbar_wait(bar_accfree, (t - 1) & 1, abort_flag, tmo, 209))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ts(tmem + C::kColDV, tmem + C::kColS + (kk >> 2) * 64 + (kk & 3) * 8,
+                     desc_at(dMN, oDO + st * TILE + kk * 2048), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
+            tc_commit(&bar_dvdone[st]);  // also dP_i: both readers of dO_i are done
+            if (it + 1 < n) {
+              // next S^T as early as possible: its softmax overlaps dQ, dK of tile it
+              if (!mbar_wait(&bar_qfull[st1], ph1, abort_flag, tmo, 214)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              bwd_issue_t<D, T>(tmem + C::kColS, dKm, oK, oQ + st1 * TILE);
+              tc_commit(bar_s);
+              // dP^T(it+1) overwrites dP^T(it), read once dS_i is written, and at
+              // d = 128 also the dQ partial, free once the drain has read it
+              if (!mbar_wait(bar_ds, g & 1, abort_flag, tmo, 215) ||
+                  (D == 128 && !mbar_wait(bar_dqfree, g & 1, abort_flag, tmo, 217)) ||
+                  !mbar_wait(&bar_dofull[st1], ph1, abort_flag, tmo, 218)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              bwd_issue_t<D, T>(tmem + C::kColDP, dKm, oV, oDO + st1 * TILE);
+              tc_commit(bar_dp);
+            }
+          }
+          if (!ok) break;
+          tc_commit(bar_final);  // this issuer's products of the item are done
+          g0_ += n;
+          ++t_;
         }
       } else {
         // dQ_i partial = dS K_j, dK += dS^T Q_i
-        bool ok = mbar_wait(bar_kv, 0, abort_flag, tmo, 224);
-        for (int it = 0; it < n && ok; ++it) {
-          const int st = it & 1;
-          if (!mbar_wait(bar_ds, it & 1, abort_flag, tmo, 225)) break;
-          tc_fence_after();
-          if (D != 128 && it > 0) {  // separate dQ columns: only the previous dQ must be drained
-            if (!mbar_wait(bar_dqfree, (it - 1) & 1, abort_flag, tmo, 216)) break;
+        bool ok = true;
+        int g0_ = 0, t_ = 0;
+        for (int wu = blockIdx.x; wu < units && ok; wu += kPersist ? static_cast<int>(gridDim.x) : units)
+        for (int half = 0; half < kHalves && ok; ++half) {
+          int j, bh, i0, n;
+          if (!unit_item(wu, half, j, bh, i0, n)) continue;
+          const int g0 = kPersist ? g0_ : 0;  // this item's first step
+          const int t = kPersist ? t_ : 0;    // items before this one
+          if (!mbar_wait(bar_kv, t & 1, abort_flag, tmo, 224)) {
+            ok = false;
+            break;
+          }
+          for (int it = 0; it < n; ++it) {
+            const int g = g0 + it;
+            const int st = g & 1;
+            if (!mbar_wait(bar_ds, g & 1, abort_flag, tmo, 225)) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
-          }
-          // dQ first (A = dS MN-major in smem, B = K_j MN-major), so that its
-          // drain overlaps dK
+            if (D != 128 && g > 0) {  // separate dQ columns: only the previous dQ must be drained
+              if (!mbar_wait(bar_dqfree, (g - 1) & 1, abort_flag, tmo, 216)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            // dQ first (A = dS MN-major in smem, B = K_j MN-major), so that its
+            // drain overlaps dK
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + C::kColDQ, desc_at(dMN, oDS + kk * 2048), desc_at(dMN, oK + kk * 2048), idesc_q,
-                   kk > 0 ? 1u : 0u);
-          tc_commit(bar_dqfull);
-          // dK += dS^T Q_i   (A = dS^T K-major in smem, B = Q_i MN-major)
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tmem + C::kColDQ, desc_at(dMN, oDS + kk * 2048), desc_at(dMN, oK + kk * 2048), idesc_q,
+                     kk > 0 ? 1u : 0u);
+            tc_commit(bar_dqfull);
+            // the item's first dK starts over once the previous item's dK is read out
+            if (it == 0 && t > 0) {
+              if (!mbar_wait(bar_accfree, (t - 1) & 1, abort_flag, tmo, 226)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            // dK += dS^T Q_i   (A = dS^T K-major in smem, B = Q_i MN-major)
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t offa = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_ss(tmem + C::kColDK, desc_at(dKm, oDS + offa), desc_at(dMN, oQ + st * TILE + kk * 2048),
-                   idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t offa = (kk >> 2) * 16384 + (kk & 3) * 32;
+              mma_ss(tmem + C::kColDK, desc_at(dKm, oDS + offa), desc_at(dMN, oQ + st * TILE + kk * 2048),
+                     idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
+            }
+            tc_commit(bar_dsfree);
+            tc_commit(&bar_qempty[st]);
           }
-          tc_commit(bar_dsfree);
-          tc_commit(&bar_qempty[st]);
+          if (!ok) break;
+          tc_commit(bar_final);  // this issuer's products of the item are done
+          g0_ += n;
+          ++t_;
         }
       }
-      tc_commit(bar_final);
       tc_commit(bar_drain);
       drain_wait(bar_drain, 0, 219);
     }
@@ -330,7 +467,6 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
     // ------------------------------------------------------------ compute
     const int h = warp >> 2;  // query-column half
     const int wq = warp & 3;
-    const int key = j * 128 + wq * 32 + lane;  // epilogue: this thread's key row
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     // Scores, dP and P are read and written in the 16-lane fragment layout:
     // thread t holds key rows 32wq + 16b + 8rr + t/4 (b, rr in {0, 1}) and, in
@@ -341,18 +477,29 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
     const uint32_t tS = tmem + lane_off + C::kColS + 64 * h;
     const uint32_t tDP = tmem + lane_off + C::kColDP + 64 * h;
     const float c = p.scale_log2;
-    int pad = 0;  // bit 2b+rr: that key row is padding
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (j * 128 + 32 * wq + 8 * q + g4 >= N) pad |= 1 << q;
     // dS tile: K-major, row = key, 128-byte swizzle (16-byte unit u of row k at
     // unit u ^ (k & 7)); stmatrix row address of this lane for block b, group g
     const uint32_t ds_lane = smem_u32(sDS) + h * 16384 + (32 * wq + (lane & 15)) * 128;
     const uint32_t ds_sw = lane & 7;
     bool ok = true;
+    int g0_ = 0, t_ = 0;
+    for (int wu = blockIdx.x; wu < units && ok; wu += kPersist ? static_cast<int>(gridDim.x) : units)
+    for (int half = 0; half < kHalves && ok; ++half) {
+    // only the step count and the padding bits stay live through the steps
+    int n, pad = 0;  // pad bit 2b+rr: that key row is padding
+    {
+      int j, bh, i0;
+      if (!unit_item(wu, half, j, bh, i0, n)) continue;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (j * 128 + 32 * wq + 8 * q + g4 >= N) pad |= 1 << q;
+    }
+    const int g0 = kPersist ? g0_ : 0;  // this item's first step
+    const int t = kPersist ? t_ : 0;    // items before this one
     for (int it = 0; it < n; ++it) {
-      const int st = it & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_s, it & 1, abort_flag, tmo, 220))) {
+      const int g = g0 + it;
+      const int st = g & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_s, g & 1, abort_flag, tmo, 220))) {
         ok = false;
         break;
       }
@@ -427,11 +574,11 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
 #pragma unroll
       for (int g = 0; g < 8; ++g) dvv[g] = dv2[4 * g];
 
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_dp, it & 1, abort_flag, tmo, 221))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_dp, g & 1, abort_flag, tmo, 221))) {
         ok = false;
         break;
       }
-      if (it > 0 && !__all_sync(0xffffffffu, mbar_wait(bar_dsfree, (it - 1) & 1, abort_flag, tmo, 222))) {
+      if (g > 0 && !__all_sync(0xffffffffu, mbar_wait(bar_dsfree, (g - 1) & 1, abort_flag, tmo, 222))) {
         ok = false;
         break;
       }
@@ -463,9 +610,18 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       tc_fence_before();
       mbar_arrive(bar_ds);
     }
-    // epilogue: half 0 writes dK (times scale), half 1 writes dV
-    if (ok && __all_sync(0xffffffffu, mbar_wait(bar_final, 0, abort_flag, tmo, 223))) {
+    if (!ok) break;
+    // epilogue: half 0 writes dK (times scale), half 1 writes dV; the
+    // accumulators are handed back once read
+    if (!__all_sync(0xffffffffu, mbar_wait(bar_final, t & 1, abort_flag, tmo, 223))) {
+      ok = false;
+      break;
+    }
+    {
       tc_fence_after();
+      int j, bh, i0, n_;
+      unit_item(wu, half, j, bh, i0, n_);
+      const int key = j * 128 + wq * 32 + lane;  // this thread's key row
       const bool key_ok = key < N;
       const uint32_t tAcc = tmem + lane_off + (h == 0 ? C::kColDK : C::kColDV);
       const float mul = (h == 0) ? p.scale : 1.0f;
@@ -485,6 +641,11 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
           for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
         }
       }
+      tc_fence_before();
+      mbar_arrive(bar_accfree);
+    }
+    g0_ += n;
+    ++t_;
     }
   } else {
     setmaxnreg_inc<C::kRegsDrain>();
@@ -499,9 +660,20 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
     const int wq = warp & 3;
     const uint32_t tQ = tmem + (static_cast<uint32_t>(wq * 32) << 16) + C::kColDQ;
     const uint32_t swz = static_cast<uint32_t>(lane & 7);
+    bool ok = true;
+    int g0_ = 0;
+    for (int wu = blockIdx.x; wu < units && ok; wu += kPersist ? static_cast<int>(gridDim.x) : units)
+    for (int half = 0; half < kHalves && ok; ++half) {
+    int j, bh, i0, n;
+    if (!unit_item(wu, half, j, bh, i0, n)) continue;
+    const int g0 = kPersist ? g0_ : 0;  // this item's first step
     for (int it = 0; it < n; ++it) {
-      const int st = it & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_dqfull, it & 1, abort_flag, tmo, 230))) break;
+      const int g = g0 + it;
+      const int st = g & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_dqfull, g & 1, abort_flag, tmo, 230))) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       uint8_t* stage = (D == 128 ? sDO + st * TILE : smem + C::kOffStage) + wq * 8192;
       uint8_t* my_row = stage + lane * 128;
@@ -519,7 +691,10 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
       mbar_arrive(bar_dqfree);
       // dV_i and dP_i have read dO_i: its buffer may take the staging, and
       // be handed back to the producer afterwards
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar_dvdone[st], (it >> 1) & 1, abort_flag, tmo, 232))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar_dvdone[st], (g >> 1) & 1, abort_flag, tmo, 232))) {
+        ok = false;
+        break;
+      }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         *reinterpret_cast<uint4*>(my_row + ((u ^ swz) << 4)) = make_uint4(a[4 * u], a[4 * u + 1], a[4 * u + 2], a[4 * u + 3]);
@@ -556,6 +731,8 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
         mbar_arrive(&bar_doempty[st]);  // the producer may load the next dO into this stage
       }
       __syncwarp();
+    }
+    g0_ += n;
     }
     if (lane == 0) bulk_wait_group0();  // the additions have reached global memory
     __syncwarp();

@@ -165,12 +165,12 @@ bool ensure_smem_attr(K kernel, int bytes) {
 // The backward kernel rebalances registers between warpgroups (setmaxnreg);
 // the split is only safe for a compiled register count in [kRegsMin, kRegsMax],
 // so a build outside that range is refused before its first launch.
-template <int D, typename T>
+template <int D, typename T, bool kPersist>
 bool bwd_regs_ok(int dev) {
   static std::atomic<int> checked[kMaxDevices];  // one table per kernel instantiation
   if (checked[dev].load(std::memory_order_acquire)) return true;
   cudaFuncAttributes a{};
-  if (cudaFuncGetAttributes(&a, exattn::attn_bwd_kernel<D, T>) != cudaSuccess) return false;
+  if (cudaFuncGetAttributes(&a, exattn::attn_bwd_kernel<D, T, kPersist>) != cudaSuccess) return false;
   if (a.numRegs < exattn::BwdCfg<D>::kRegsMin || a.numRegs > exattn::BwdCfg<D>::kRegsMax) return false;
   checked[dev].store(1, std::memory_order_release);
   return true;
@@ -513,6 +513,18 @@ int preprocess_impl(const void* o, const void* dO, const float* lse, int B, int 
   return launch_status();
 }
 
+// Key tiles per head up to which the main backward runs persistent CTAs.
+constexpr int kBwdPersistMaxTiles = 8;
+
+template <int D, typename T, bool kPersist>
+int launch_bwd(const BwdParams& p, dim3 grid, int dev, cudaStream_t s) {
+  constexpr int smem = exattn::BwdCfg<D>::kSmem;
+  if (!bwd_regs_ok<D, T, kPersist>(dev)) return ATTN_ERR_LAUNCH;
+  if (!ensure_smem_attr(exattn::attn_bwd_kernel<D, T, kPersist>, smem)) return ATTN_ERR_LAUNCH;
+  exattn::attn_bwd_kernel<D, T, kPersist><<<grid, exattn::BwdCfg<D>::kThreads, smem, s>>>(p);
+  return launch_status();
+}
+
 template <typename T>
 int dkdv_impl(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, int B, int H,
                   int N, int d, float scale, int causal, void* workspace, size_t workspace_bytes_given,
@@ -550,20 +562,21 @@ int dkdv_impl(const void* q, const void* k, const void* v, const void* dO, void*
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
   p.debug_flags = g_debug_flags.load(std::memory_order_relaxed);
-  const dim3 grid(static_cast<unsigned>(p.ntiles) * static_cast<unsigned>(BH));
+  // Up to kBwdPersistMaxTiles key tiles per head (N <= 1024), where a CTA's
+  // start-up and epilogue are a large share of its few steps: persistent
+  // CTAs, one per SM (the kernel's TMEM and shared memory allow no second),
+  // each walking the work units (a key tile, or under the causal mask a pair
+  // of key tiles, of one head) with a stride of the grid.  Longer rows: one
+  // CTA per key tile, handed out by the hardware as SMs free up (measured
+  // faster there).
+  const bool persist = p.ntiles <= kBwdPersistMaxTiles;
+  p.paired = (persist && causal) ? 1 : 0;
+  const long long units = static_cast<long long>(p.paired ? (p.ntiles + 1) / 2 : p.ntiles) * BH;
+  const dim3 grid(static_cast<unsigned>(persist ? std::min<long long>(units, sm_count()) : units));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 64) {
-    constexpr int smem = exattn::BwdCfg<64>::kSmem;
-    if (!(bwd_regs_ok<64, T>(dev))) return ATTN_ERR_LAUNCH;
-    if (!ensure_smem_attr(exattn::attn_bwd_kernel<64, T>, smem)) return ATTN_ERR_LAUNCH;
-    exattn::attn_bwd_kernel<64, T><<<grid, exattn::BwdCfg<64>::kThreads, smem, s>>>(p);
-  } else {
-    constexpr int smem = exattn::BwdCfg<128>::kSmem;
-    if (!(bwd_regs_ok<128, T>(dev))) return ATTN_ERR_LAUNCH;
-    if (!ensure_smem_attr(exattn::attn_bwd_kernel<128, T>, smem)) return ATTN_ERR_LAUNCH;
-    exattn::attn_bwd_kernel<128, T><<<grid, exattn::BwdCfg<128>::kThreads, smem, s>>>(p);
-  }
-  return launch_status();
+  if (d == 64)
+    return persist ? launch_bwd<64, T, true>(p, grid, dev, s) : launch_bwd<64, T, false>(p, grid, dev, s);
+  return persist ? launch_bwd<128, T, true>(p, grid, dev, s) : launch_bwd<128, T, false>(p, grid, dev, s);
 }
 
 template <typename T>

@@ -53,10 +53,11 @@ def _kernel(regs, stem, d, params, elem, flag=None):
     return regs[name]
 
 
+@pytest.mark.parametrize("persist", [False, True])
 @pytest.mark.parametrize("elem", ELEMS)
 @pytest.mark.parametrize("d", [64, 128])
-def test_backward_register_split_fits(registers, d, elem):
-    r = _kernel(registers, "attn_bwd_kernel", d, "BwdParams", elem)
+def test_backward_register_split_fits(registers, d, elem, persist):
+    r = _kernel(registers, "attn_bwd_kernel", d, "BwdParams", elem, flag=persist)
     threads = _const("bwd.cuh", "kThreads")
     drain, side = _const("bwd.cuh", "kRegsDrain"), _const("bwd.cuh", "kRegsSide")
     # warpgroup 2 (drain) rises from r to `drain`, warpgroup 3 falls from r to `side`
