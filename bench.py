@@ -321,7 +321,7 @@ def run_ours(args, rank, world, local_rank):
                         "fwd_of_spec_2250": fwd_tf / spec_peak, "bwd_of_spec_2250": bwd_tf / spec_peak,
                         "peak_source": peak_src},
         "kernels": {k_: {"mean_ms": mean[k_]} for k_ in mean},
-        "roofline": {"kernel": "attn_bwd_kernel<128, bf16>" if dominant == "bwd_dkdv" else "attn_fwd_kernel<128, bf16>",
+        "roofline": {"kernel": "attn_bwd_kernel<128, bf16, 0>" if dominant == "bwd_dkdv" else "attn_fwd_kernel<128, bf16, 0>",
                      "bound": "tensor", "achieved": dom_tf, "peak": peak, "unit": "TFLOP/s",
                      "frac": dom_tf / peak, "peak_kind": f"bf16 burst ({peak_src})",
                      "frac_of_sustained": dom_tf / peak_sus,
