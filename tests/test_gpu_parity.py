@@ -38,6 +38,19 @@ def test_ragged_lengths(cuda_device, N, d, causal):
     check_all(got, ref, what=f"N={N} d={d} causal={causal}")
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1025, 1500, 2049, 3001, 4095])
+def test_mid_lengths(cuda_device, N, d, causal):
+    """Lengths past the short-row forward configuration (the backward runs
+    persistent CTAs up to 2048): ragged tails, odd and even numbers of query
+    blocks and key tiles, several heads."""
+    q, k, v, do = _inputs(2, 3, N, d, seed=N * 7 + d + int(causal))
+    scale = 1 / math.sqrt(d)
+    got = run_cuda(q, k, v, do, causal, scale)
+    check_all(got, oracle_ref(q, k, v, do, causal, scale), what=f"N={N} d={d} causal={causal}")
+
+
 def test_small_causal_stability_config(cuda_device):
     w = W.SMALL_CAUSAL_STABILITY
     q, k, v, do = W.make_inputs(w)
