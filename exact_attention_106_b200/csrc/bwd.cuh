@@ -156,23 +156,20 @@ __global__ void __launch_bounds__(512, 1) attn_bwd_kernel(const __grid_constant_
   const int lane = threadIdx.x & 31;
   const int N = p.N;
   const int ntq = p.ntiles;  // query tiles
-  // The CTA is persistent: it works through the items (key tile j, head bh)
-  // blockIdx.x, blockIdx.x + gridDim.x, ...  Item order: key tile 0 first
-  // (under the causal mask it sees the most query tiles), a few heads at a
-  // time.  Every role walks the same sequence; a step's rings and barriers
-  // take their phases from its index g in the CTA's whole sequence of steps,
-  // so that one item's loads and products start while the previous item's
-  // epilogue runs.
-  //
-  // The host either launches one CTA per item (each CTA then runs a single
-  // unit, and the hardware hands out the items as SMs free up), or, for
-  // short problems where a CTA's start-up and epilogue weigh, one CTA per SM
-  // with p.paired set under the causal mask.  Key tile j then sees ntq - j
-  // query tiles, so the items are taken in pairs (j, ntq - 1 - j) of one
-  // head, heavier first: every pair costs ntq + 1 steps, and a fixed stride
-  // over equal units balances the SMs as well as the hardware's scheduling
-  // would (with an odd ntq the middle tile stands alone, last in its head's
-  // order).  Otherwise every item is its own unit.
+  // Work units.  With kPersist false the CTA runs the single item blockIdx.x
+  // (key tile j, head bh), and the hardware hands out the items as SMs free
+  // up: key tile 0 first (under the causal mask it sees the most query
+  // tiles), a few heads at a time.  With kPersist (short rows, where a CTA's
+  // start-up and epilogue weigh) one CTA per SM walks the units blockIdx.x,
+  // blockIdx.x + gridDim.x, ...; under the causal mask (p.paired) a unit is
+  // the pair of key tiles (j, ntq - 1 - j) of one head, heavier first, which
+  // together see ntq + 1 query tiles, so that a fixed stride over equal units
+  // balances the SMs as well as the hardware's scheduling would (with an odd
+  // ntq the middle tile stands alone, last in its head's order).  Every role
+  // walks the same sequence; a step's rings and barriers take their phases
+  // from its index g in the CTA's whole sequence of steps (the counters are 0
+  // without kPersist), so that one item's loads and products start while the
+  // previous item's epilogue runs.
   const int npt = (ntq + 1) / 2;
   const bool paired = kPersist && p.causal && p.paired;
   constexpr int kHalves = kPersist ? 2 : 1;
