@@ -194,11 +194,10 @@ int head_group(int BH, double per_head_bytes) {
 // Launches the forward kernel for a filled-in parameter block (tensor maps
 // and sizes set by the caller).
 template <typename T>
-int launch_fwd(FwdParams& p, int d, int dev, cudaStream_t s) {
+int launch_fwd(FwdParams& p, int d, cudaStream_t s) {
   p.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
   p.debug_flags = g_debug_flags.load(std::memory_order_relaxed);
   const dim3 grid(static_cast<unsigned>(p.nblocks) * static_cast<unsigned>(p.splits) * static_cast<unsigned>(p.BH));
-  (void)dev;
   if constexpr (sizeof(T) == 1) {  // e4m3: head_dim 128 only
     if (d != 128) return ATTN_ERR_INVALID;
     constexpr int smem = exattn::FwdCfg<128, T>::kSmem;
@@ -282,7 +281,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, i
     p.nblocks = (N + 127) / 128;
     return launch_fwd_lean<T>(p, d, reinterpret_cast<cudaStream_t>(stream));
   }
-  return launch_fwd<T>(p, d, dev, reinterpret_cast<cudaStream_t>(stream));
+  return launch_fwd<T>(p, d, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // e4m3 inputs: the per-tensor descale factors fold into the score scale (Q,
@@ -320,7 +319,7 @@ int fwd_fp8_impl(const void* q, const void* k, const void* v, void* o, float* ls
   p.scale = eff;
   p.scale_log2 = eff * 1.4426950408889634f;
   p.o_mul = v_descale;
-  return launch_fwd<__nv_fp8_e4m3>(p, d, dev, reinterpret_cast<cudaStream_t>(stream));
+  return launch_fwd<__nv_fp8_e4m3>(p, d, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // ------------------------------------------------------ split-key forward
@@ -480,7 +479,7 @@ int kvsplit_impl(const void* q, const void* k, const void* v, void* o, float* ls
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o_mul = 1.0f;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (int st = lean ? launch_fwd_lean<T>(p, d, s) : launch_fwd<T>(p, d, dev, s)) return st;
+  if (int st = lean ? launch_fwd_lean<T>(p, d, s) : launch_fwd<T>(p, d, s)) return st;
   if (S == 1) return ATTN_OK;
   const long long rows = static_cast<long long>(BH) * Nq;
   const unsigned blocks = static_cast<unsigned>((rows + 7) / 8);
