@@ -211,6 +211,7 @@ def run_ours(args, rank, world, local_rank):
     w = rank_workload(W.by_name(args.workload), rank)
     B, H, N, d = w.shape
     q, k, v, do = W.make_inputs(w)
+    torch.cuda.reset_peak_memory_stats(dev)
     qd, kd, vd, dod = (x.to(dev) for x in (q, k, v, do))
     o = torch.empty_like(qd)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
@@ -251,6 +252,7 @@ def run_ours(args, rank, world, local_rank):
         t_end.record(stream)
         barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
+    peak_alloc = torch.cuda.max_memory_allocated(dev)  # inputs, outputs, workspace: linear in N
     status = ex.device_status(dev)
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
@@ -335,6 +337,7 @@ def run_ours(args, rank, world, local_rank):
         "cpu_baseline": cpu,
         "e2e": {"value": job_throughput(world, flops_step, e2e_steps, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "memory": {"peak_allocated_bytes": peak_alloc, "one_bf16_score_matrix_bytes": B * H * N * N * 2},
         "clocks": clk.summary(),
         "gpu_launches": 4 * args.steps,
     }

@@ -22,7 +22,7 @@ import torch
 from . import _lib
 
 __all__ = ["forward", "backward", "forward_fp8", "forward_kvsplit", "kvsplit_plan", "forward_backward_host", "bwd_workspace_bytes", "host_buffer_bytes",
-           "device_status", "ExattnError"]
+           "device_status", "set_wait_timeout_ns", "ExattnError"]
 
 ExattnError = _lib.ExattnError
 
@@ -230,6 +230,15 @@ def forward_backward_host(q, k, v, do, out, causal: bool = False, scale: Optiona
             dv.data_ptr(), B, H, N, d, _scale(d, scale), int(causal), buf.data_ptr(), buf.numel(),
             int(heads_per_chunk), _stream(dev)))
     return out
+
+
+def set_wait_timeout_ns(ns: int) -> None:
+    """Limit of every device-side wait of the library's kernels, in ns (0
+    restores the default of one second).  The environment variable
+    EXATTN_WAIT_TIMEOUT_NS sets it when the library is loaded."""
+    if ns < 0:
+        raise ValueError("the wait limit must be >= 0")
+    _lib.load().attn_set_wait_timeout_ns(int(ns))
 
 
 def device_status(device=None) -> int:

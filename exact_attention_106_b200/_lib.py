@@ -64,6 +64,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
             fn = getattr(lib, name)
             fn.restype = res
             fn.argtypes = args
+        env = os.environ.get("EXATTN_WAIT_TIMEOUT_NS")
+        if env:  # the limit of every device-side wait, in ns (a malformed value raises ValueError)
+            ns = int(env)
+            if ns < 0:
+                raise ValueError("EXATTN_WAIT_TIMEOUT_NS must be >= 0")
+            lib.attn_set_wait_timeout_ns(ns)
         _lib = lib
     return _lib
 

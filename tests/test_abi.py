@@ -160,3 +160,16 @@ def test_kvsplit_plan_is_per_whole_tile(lib):
             plans = {lib.attn_fwd_kvsplit_count(B, H, Nq, nk, 128, 1, 0) for nk in range(128 * t0 + 1, 128 * (t0 + 1) + 1)}
             assert len(plans) == 1, (B, H, Nq, t0, plans)
             assert 1 <= plans.pop() <= 64
+
+
+def test_wait_limit_from_the_environment():
+    """EXATTN_WAIT_TIMEOUT_NS sets the device-side wait limit when the library
+    loads; a malformed or negative value is refused rather than ignored."""
+    import subprocess
+    import sys
+    code = "import exact_attention_106_b200._lib as L; L.load()"
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    for val, ok in (("5000000", True), ("0", True), ("abc", False), ("-1", False)):
+        r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True,
+                           env=dict(os.environ, EXATTN_WAIT_TIMEOUT_NS=val))
+        assert (r.returncode == 0) == ok, (val, r.stderr[-300:])
