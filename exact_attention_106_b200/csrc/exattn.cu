@@ -512,11 +512,15 @@ int preprocess_impl(const void* o, const void* dO, const float* lse, int B, int 
   return launch_status();
 }
 
-// Key tiles per head up to which the main backward runs persistent CTAs:
-// 8 (N <= 1024), and 16 (N <= 2048) under the causal mask or at head_dim 64
-// (measured: +3 to +14% there; -1% for 16 tiles of d = 128 without the mask).
-constexpr int kBwdPersistMaxTiles = 8;
-constexpr int kBwdPersistMaxTilesCausalOrD64 = 16;
+// Key tiles per head up to which the main backward runs persistent CTAs
+// (measured against one CTA per key tile): at head_dim 128, 8 (N <= 1024;
+// +10 to +14%) and 16 under the causal mask (+3%; -1% without it); at
+// head_dim 64, 32 (+1 to +4%) and 64 under the causal mask (+2%; -0.5%
+// without it).
+bool bwd_persistent(int ntiles, int d, int causal) {
+  if (d == 64) return ntiles <= (causal ? 64 : 32);
+  return ntiles <= (causal ? 16 : 8);
+}
 
 template <int D, typename T, bool kPersist>
 int launch_bwd(const BwdParams& p, dim3 grid, int dev, cudaStream_t s) {
@@ -564,15 +568,14 @@ int dkdv_impl(const void* q, const void* k, const void* v, const void* dO, void*
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
   p.debug_flags = g_debug_flags.load(std::memory_order_relaxed);
-  // Short rows (see kBwdPersistMaxTiles), where a CTA's start-up and
+  // Short rows (see bwd_persistent), where a CTA's start-up and
   // epilogue are a large share of its few steps: persistent
   // CTAs, one per SM (the kernel's TMEM and shared memory allow no second),
   // each walking the work units (a key tile, or under the causal mask a pair
   // of key tiles, of one head) with a stride of the grid.  Longer rows: one
   // CTA per key tile, handed out by the hardware as SMs free up (measured
   // faster there).
-  const bool persist = p.ntiles <= kBwdPersistMaxTiles ||
-                       (p.ntiles <= kBwdPersistMaxTilesCausalOrD64 && (causal || d == 64));
+  const bool persist = bwd_persistent(p.ntiles, d, causal);
   p.paired = (persist && causal) ? 1 : 0;
   const long long units = static_cast<long long>(p.paired ? (p.ntiles + 1) / 2 : p.ntiles) * BH;
   const dim3 grid(static_cast<unsigned>(persist ? std::min<long long>(units, sm_count()) : units));
