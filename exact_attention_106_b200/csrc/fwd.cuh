@@ -355,14 +355,14 @@ __global__ void __launch_bounds__(FwdCfg<D, T, kLean>::kThreads, FwdCfg<D, T, kL
         for (int i = 0; i < 128; ++i)
           if (i > lim) sr[i] = __float_as_uint(-INFINITY);
       }
-      // row maximum: four independent chains of 3-input max
-      float mxa[4];
+      // row maximum: eight independent chains of 3-input max
+      float mxa[8];
 #pragma unroll
-      for (int t = 0; t < 4; ++t) mxa[t] = __uint_as_float(sr[t]);
+      for (int t = 0; t < 8; ++t) mxa[t] = __uint_as_float(sr[t]);
 #pragma unroll
-      for (int i = 4; i < 128; i += 2)
-        mxa[(i >> 1) & 3] = max3f(mxa[(i >> 1) & 3], __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]));
-      const float mx = fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3]));
+      for (int i = 8; i < 128; i += 2)
+        mxa[(i >> 1) & 7] = max3f(mxa[(i >> 1) & 7], __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]));
+      const float mx = fmaxf(max3f(mxa[0], mxa[1], mxa[2]), max3f(mxa[3], mxa[4], max3f(mxa[5], mxa[6], mxa[7])));
       const float m_new = (mx > m_ref + thr) ? mx : m_ref;
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
       const float alpha = ex2((m_ref - m_use) * c);
