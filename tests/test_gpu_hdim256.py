@@ -55,10 +55,11 @@ def test_hdim256_bench_workload_sampled_heads(cuda_device):
 
 
 @pytest.mark.parametrize("nq,nk,splits", [(1, 5000, 0), (16, 3000, 3), (1000, 1000, 4)])
-def test_hdim256_kvsplit(cuda_device, nq, nk, splits):
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16], ids=["bf16", "fp16"])
+def test_hdim256_kvsplit(cuda_device, nq, nk, splits, dtype):
     g = torch.Generator().manual_seed(nq + nk)
-    q = torch.randn((1, 2, nq, 256), generator=g).bfloat16()
-    k, v = (torch.randn((1, 2, nk, 256), generator=g).bfloat16() for _ in range(2))
+    q = torch.randn((1, 2, nq, 256), generator=g).to(dtype)
+    k, v = (torch.randn((1, 2, nk, 256), generator=g).to(dtype) for _ in range(2))
     for causal in (False, True):
         o, lse = ex.forward_kvsplit(q.to(cuda_device), k.to(cuda_device), v.to(cuda_device), causal=causal,
                                     splits=splits)
